@@ -1,0 +1,363 @@
+#!/usr/bin/env python
+"""Benchmark of the SSD forward pass on the Mamba-2 2.7B-shaped layer.
+
+Workload: B=4, L=4096, H=80 heads, P=64, N=128, G=1, chunk 256, bf16 I/O,
+seeded synthetic inputs (selective_state_space_17_b200.inputs). A step is one
+ssd_forward call over the whole batch (all steps of the chunked algorithm).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line on rank 0. ``value`` is Mtokens/s over all ranks (tokens
+= B*L per rank per step; every rank runs its own copy of the layer: the work
+shards by batch and head with no data-path collective, so scaling is weak).
+Timing: CUDA events on the launching stream around each step, L2 flushed
+(256 MiB write) between steps outside the events, max over ranks.
+``--impl reference`` times the fp64 CPU oracle on the host cores instead
+(rank 0 only), on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from selective_state_space_17_b200 import inputs as gen  # noqa: E402
+
+METRIC = "SSD fwd Mtokens/s per layer on 1 B200; % of HBM/tensor-core roofline"
+UNIT = "Mtokens/s"
+WORKLOAD = gen.LAYER_2P7B
+L2_FLUSH_BYTES = 256 << 20
+
+
+def compulsory_bytes(w: gen.Workload) -> int:
+    """x and y in the I/O dtype, dt, Bm and Cm once per group, final_state,
+    A and D: every byte the layer must read or write at least once."""
+    es = 2 if w.dtype == "bf16" else 4
+    BL = w.B * w.L
+    return (2 * BL * w.H * w.P * es + BL * w.H * 4 + 2 * BL * w.G * w.N * es
+            + w.B * w.H * w.P * w.N * 4 + 2 * w.H * 4)
+
+
+def algorithmic_flops(w: gen.Workload) -> int:
+    """Per token and head: Q*P (causal half of the chunk's masked product with
+    X) + 4*N*P (chunk states and the state read-out); per token and group:
+    Q*N (causal half of C B^T)."""
+    BL = w.B * w.L
+    return BL * w.H * (w.chunk * w.P + 4 * w.N * w.P) + BL * w.G * w.chunk * w.N
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        self.out.flush()
+        rows = []
+        with open(self.out.name) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(dict(sm=float(parts[1]), max=float(parts[2]),
+                                     power=float(parts[3]) if parts[3] not in ("[N/A]", "") else 0.0,
+                                     hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+                except ValueError:
+                    continue
+        os.unlink(self.out.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"]}
+        reasons = set()
+        for r in rows:
+            if r["hw"] == "Active":
+                reasons.add("hw_slowdown")
+            if r["hwt"] == "Active":
+                reasons.add("hw_thermal_slowdown")
+            if r["swt"] == "Active":
+                reasons.add("sw_thermal_slowdown")
+            if r["pcap"] == "Active":
+                reasons.add("sw_power_cap")
+        loaded = [r["sm"] for r in rows if r["power"] > 200.0] or [r["sm"] for r in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r["max"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+def time_oracle_sample(w: gen.Workload, inp, heads: int, min_seconds: float):
+    """Run the fp64 oracle on batch row 0, the first `heads` heads (their
+    groups whole), full sequence; repeat until min_seconds. Returns
+    (Mtokens/s-equivalent, threads, sample description, seconds)."""
+    import oracle
+    hpg = w.H // w.G
+    heads = max(hpg, (heads // hpg) * hpg)
+    x, dt, A, Bm, Cm, D = inp.f64(0, 1, heads=(0, heads))
+    threads = min(oracle.default_threads(), heads)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.forward(x, dt, A, Bm, Cm, D, nthreads=threads)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds:
+            break
+    tokens_equiv = reps * w.L * heads / w.H  # a full-layer token needs all H heads
+    sample = (f"batch row 0 of {w.B}, heads 0..{heads - 1} of {w.H}, all {w.L} tokens, "
+              f"{reps} run(s); tokens counted as L*heads/H")
+    return tokens_equiv / el / 1e6, threads, sample, el
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = WORKLOAD
+    inp = w.make(0)
+    per_step = []
+    info = None
+    for i in range(args.warmup + args.steps):
+        v, threads, sample, el = time_oracle_sample(w, inp, heads=8, min_seconds=0.0)
+        if i >= args.warmup:
+            per_step.append(el)
+            info = (threads, sample)
+    tokens_equiv = w.L * 8 / w.H
+    ms = statistics.mean(per_step) * 1e3
+    value = tokens_equiv / (ms / 1e3) / 1e6
+    threads, sample = info
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": w.name, "global_batch": w.B, "seq_len": w.L,
+                                        "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": "per step: " + sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from selective_state_space_17_b200 import ssd
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: WORLD_SIZE={world} but --gpus {args.gpus}", file=sys.stderr)
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    w = WORKLOAD
+    inp = w.make(seed=rank)
+    code = ssd.SSD_BF16 if w.dtype == "bf16" else ssd.SSD_F32
+
+    def io(a):
+        if w.dtype == "bf16":
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+        return torch.from_numpy(a)
+
+    host = dict(x=io(inp.x), dt=torch.from_numpy(inp.dt), A=torch.from_numpy(inp.A),
+                Bm=io(inp.Bm), Cm=io(inp.Cm), D=torch.from_numpy(inp.D))
+    d = {k: v.to(dev) for k, v in host.items()}
+    y = torch.empty_like(d["x"])
+    fs = torch.empty((w.B, w.H, w.P, w.N), dtype=torch.float32, device=dev)
+    ws = torch.zeros(ssd.workspace_size(w.B, w.L, w.H, w.P, w.G, w.N, w.chunk, code),
+                     dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ssd.forward(d["x"], d["dt"], d["A"], d["Bm"], d["Cm"], d["D"], chunk=w.chunk, y=y,
+                    final_state=fs, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    ssd.poll_status(stream)
+    barrier()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        barrier()
+    ssd.poll_status(stream)
+    per_step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms_local = statistics.mean(per_step_ms)
+    t = torch.tensor([ms_local], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    tokens_all = w.tokens * world
+    value = tokens_all / (ms / 1e3) / 1e6
+
+    # end to end through the host-buffer entry point: H2D inputs, forward, D2H y + state
+    pin = {k: v.pin_memory() for k, v in host.items()}
+    y_host = torch.empty_like(host["x"]).pin_memory()
+    fs_host = torch.empty((w.B, w.H, w.P, w.N), dtype=torch.float32).pin_memory()
+    dbuf = torch.zeros(ssd.forward_host_buffer_size(w.B, w.L, w.H, w.P, w.G, w.N, w.chunk, code),
+                       dtype=torch.uint8, device=dev)
+    e2e_steps = max(3, min(args.steps, 10))
+
+    def e2e_step():
+        ssd.forward_host(pin["x"], pin["dt"], pin["A"], pin["Bm"], pin["Cm"], pin["D"], y_host,
+                         fs_host, chunk=w.chunk, device_buffer=dbuf, stream=stream)
+
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e_end.record(stream)
+    barrier()
+    e2e_ms = e_start.elapsed_time(e_end) / e2e_steps
+    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_ms = float(t.item())
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = y_host.numel() * y_host.element_size() + fs_host.numel() * 4
+
+    hbm_peak, tc_peak, peak_kind = measured_peaks()
+    nbytes = compulsory_bytes(w)
+    flops = algorithmic_flops(w)
+    kernel_ms = ms  # one ssd_forward call: its kernels back to back
+    achieved_gbs = nbytes / (kernel_ms / 1e3) / 1e9
+    achieved_tflops = flops / (kernel_ms / 1e3) / 1e12
+    t_hbm = nbytes / (hbm_peak * 1e9)
+    t_tc = flops / (tc_peak * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    launches = ssd.kernel_count(w.B, w.L, w.H, w.P, w.G, w.N, w.chunk, code)
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        try:
+            with open(tpath) as f:
+                traffic = json.load(f).get(w.name)
+        except (OSError, ValueError):
+            traffic = None
+
+    result = None
+    if rank == 0:
+        result = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic (seeded; see inputs.py)",
+            "config": {"workload": w.name, "global_batch": w.B * world, "seq_len": w.L,
+                       "heads": w.H, "headdim": w.P, "d_state": w.N, "groups": w.G,
+                       "chunk": w.chunk, "parallelism": f"replicas x{world} (batch/head shards)",
+                       "l2": "flushed between steps (256 MiB write, outside the events)"},
+            "roofline": {"bound": bound, "achieved": achieved_gbs if bound == "hbm" else achieved_tflops,
+                         "peak": hbm_peak if bound == "hbm" else tc_peak,
+                         "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
+                         "frac": (achieved_gbs / hbm_peak) if bound == "hbm" else (achieved_tflops / tc_peak),
+                         "traffic": traffic, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)"
+                         if peak_kind == "measured" else "fallback",
+                         "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
+                         "achieved_tflops": achieved_tflops,
+                         "roofline_ms": max(t_hbm, t_tc) * 1e3,
+                         "roofline_frac": max(t_hbm, t_tc) * 1e3 / kernel_ms},
+            "clocks": clk.summary(),
+            "e2e": {"value": tokens_all / (e2e_ms / 1e3) / 1e6, "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms, "api": "ssd_forward_host (pinned host buffers)"},
+            "gpu_launches": launches * args.steps,
+            "per_step_ms": {"min": min(per_step_ms), "median": statistics.median(per_step_ms),
+                            "max": max(per_step_ms)},
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            v, threads, sample, el = time_oracle_sample(w, inp, heads=16, min_seconds=10.0)
+            result["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads,
+                                      "kind": "oracle", "sample": sample,
+                                      "seconds": round(el, 2)}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if result is not None:
+        print(json.dumps(result), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps, reported as run
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

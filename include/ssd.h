@@ -1,0 +1,146 @@
+/*
+ * ssd.h — C ABI of the B200-native Mamba-2 SSD layer library (libssd_b200.so).
+ *
+ * The operation. Per batch b and head h, with scalar A_h < 0, step sizes
+ * dt[b,t,h] >= 0, group g = h / (H / G) and a P x N state starting at zero
+ * (or at initial_state):
+ *
+ *     a_t = exp(dt_t * A_h)
+ *     s_t = a_t * s_{t-1} + dt_t * x_t B_t^T          (x_t in R^P, B_t in R^N)
+ *     y_t = s_t C_t + D_h * x_t
+ *
+ * which equals Y = (L o C B^T)(dt o X) + D X with L_ij = a_i * ... * a_{j+1}
+ * for i >= j ("Mamba-2", docsaid.org, sections "Writing the SSM as one matrix"
+ * and "Simplifying A to one number"; "Mamba-2 SSD note", 0h-n0.github.io,
+ * section "SSD layer: equivalence under the scalar constraint"). The forward
+ * pass evaluates it chunk by chunk: the quadratic form inside each chunk of
+ * `chunk` tokens, the recurrence across chunks ("Mamba-2", section "Half of
+ * each route"; "Mamba-2 SSD note", section "Chunked algorithm"). The decode
+ * step applies the recurrence to one token ("Mamba-2", section "Computing
+ * with four tokens", the recurrent route for generation). The discretisation
+ * a = exp(dt A), B-bar = dt B is that of the simplified selective scan in
+ * "Mamba paper review" (youngju.dev), section 3.3.
+ *
+ * Conventions shared by every entry point:
+ *   - Tensors are dense, row-major, contiguous, in device memory unless the
+ *     name says host. x, Bm, Cm, y are in the I/O dtype (`ssd_dtype`); dt, A,
+ *     D, state, initial_state and final_state are always fp32.
+ *   - The caller owns every buffer, including the workspace. The library
+ *     allocates no device memory on these paths.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream). Argument errors are returned before anything
+ *     is enqueued. A launch failure returns SSD_ERR_CUDA.
+ *   - Device-side waits are bounded. When one gives up, the kernel records a
+ *     device status word and returns; ssd_poll_status() reports it as
+ *     SSD_ERR_TIMEOUT. Results of that call are then undefined.
+ *   - dt >= 0 and A <= 0 are the caller's contract (the decay is then in
+ *     [0, 1]); they are not checked on the device.
+ */
+#ifndef SSD_B200_H
+#define SSD_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* ssd_stream_t; /* same object as cudaStream_t */
+
+typedef enum {
+    SSD_OK = 0,
+    SSD_ERR_INVALID_ARG = 1,  /* null pointer, negative or inconsistent size */
+    SSD_ERR_UNSUPPORTED = 2,  /* valid, but a size this build does not handle */
+    SSD_ERR_MISALIGNED = 3,   /* a pointer is not 16-byte aligned */
+    SSD_ERR_CUDA = 4,         /* a CUDA call failed (launch or copy) */
+    SSD_ERR_TIMEOUT = 5,      /* a bounded device-side wait gave up */
+    SSD_ERR_WORKSPACE = 6     /* workspace null or smaller than ssd_workspace_size() */
+} ssd_status;
+
+typedef enum {
+    SSD_F32 = 0,   /* x, Bm, Cm, y in fp32: SIMT fp32 path (|rel err| ~1e-6) */
+    SSD_BF16 = 1   /* x, Bm, Cm, y in bf16: tensor-core path, fp32 accumulate */
+} ssd_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* ssd_status_string(ssd_status status);
+
+/* Bytes of device workspace ssd_forward needs for these sizes (0 if the sizes
+ * are invalid). The workspace must be zero-filled once before its first use
+ * (e.g. cudaMemset); every call leaves its control words zeroed again, so a
+ * workspace can be reused by later calls on the same stream without clearing.
+ * Two calls that run concurrently must not share one workspace. */
+size_t ssd_workspace_size(int B, int L, int H, int P, int G, int N, int chunk, ssd_dtype dtype);
+
+/*
+ * ssd_forward — chunked SSD forward pass (prefill / training forward).
+ *   x        [B, L, H, P]  I/O dtype
+ *   dt       [B, L, H]     fp32, step sizes after the softplus (>= 0)
+ *   A        [H]           fp32, per-head decay rate (<= 0)
+ *   Bm, Cm   [B, L, G, N]  I/O dtype, shared by the H/G heads of a group
+ *   D        [H]           fp32, skip term; NULL means 0
+ *   initial_state [B, H, P, N] fp32 state before token 0; NULL means zero
+ *   y        [B, L, H, P]  I/O dtype, output (bf16 outputs are rounded to
+ *                          nearest even from fp32)
+ *   final_state [B, H, P, N] fp32 state after token L-1; NULL to skip
+ *   chunk    tokens per chunk, 1..256
+ *   Sizes: B, L >= 0 (B*L == 0 is a no-op apart from final_state =
+ *   initial_state or 0), H >= 1, G >= 1, H % G == 0, P in [1, 256],
+ *   N in [1, 256]. All pointers 16-byte aligned.
+ *   The tensor-core path is taken for bf16 with P == 64, N % 16 == 0,
+ *   16 <= N <= 256, chunk in {128, 256}, H % G == 0 and every row stride a
+ *   multiple of 16 bytes; other valid sizes run the SIMT path.
+ */
+ssd_status ssd_forward(const void* x, const float* dt, const float* A, const void* Bm,
+                       const void* Cm, const float* D, const float* initial_state, void* y,
+                       float* final_state, int B, int L, int H, int P, int G, int N,
+                       int chunk, ssd_dtype dtype, void* workspace, size_t workspace_bytes,
+                       ssd_stream_t stream);
+
+/*
+ * ssd_forward_host — the same forward pass on HOST buffers (pinned memory
+ * gives asynchronous copies). Copies the inputs into `device_buffer`, runs
+ * ssd_forward on `stream`, copies y (and final_state if non-NULL) back, and
+ * synchronises `stream` before returning. `device_buffer` must hold at least
+ * ssd_forward_host_buffer_size() bytes and be zero-filled before first use.
+ */
+size_t ssd_forward_host_buffer_size(int B, int L, int H, int P, int G, int N, int chunk,
+                                    ssd_dtype dtype);
+ssd_status ssd_forward_host(const void* x_host, const float* dt_host, const float* A_host,
+                            const void* Bm_host, const void* Cm_host, const float* D_host,
+                            const float* initial_state_host, void* y_host,
+                            float* final_state_host, int B, int L, int H, int P, int G,
+                            int N, int chunk, ssd_dtype dtype, void* device_buffer,
+                            size_t device_buffer_bytes, ssd_stream_t stream);
+
+/*
+ * ssd_step — one decode step for a batch of sequences (one token each).
+ *   x [B, H, P] I/O dtype; dt [B, H] fp32; A [H] fp32; Bm, Cm [B, G, N] I/O
+ *   dtype; D [H] fp32 or NULL; state [B, H, P, N] fp32, updated in place;
+ *   y [B, H, P] I/O dtype. Sizes as for ssd_forward (L is 1).
+ */
+ssd_status ssd_step(const void* x, const float* dt, const float* A, const void* Bm,
+                    const void* Cm, const float* D, float* state, void* y, int B, int H,
+                    int P, int G, int N, ssd_dtype dtype, ssd_stream_t stream);
+
+/* Number of kernels one ssd_forward call with these sizes enqueues (0 if the
+ * sizes are invalid or there are no tokens). Host-side query; no CUDA call. */
+int ssd_forward_kernel_count(int B, int L, int H, int P, int G, int N, int chunk,
+                             ssd_dtype dtype);
+
+/* Synchronises `stream`, then reports and clears the device status word:
+ * SSD_OK, SSD_ERR_TIMEOUT (a bounded wait gave up in an earlier call), or
+ * SSD_ERR_CUDA (a CUDA error was pending on the stream). */
+ssd_status ssd_poll_status(ssd_stream_t stream);
+
+/* Test hook: sets the iteration limit of every device-side wait (0 restores
+ * the default). A limit of 1 makes a wait that is not already satisfied give
+ * up at once, which exercises the timeout path without hanging anything. */
+void ssd_set_wait_limit(uint64_t iterations);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_B200_H */

@@ -1,0 +1,91 @@
+// common.cuh — shared device helpers of the SSD library (I/O types, status word).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/ssd.h"
+
+namespace ssd {
+
+// Device status word: 0 = fine, otherwise the code of the first bounded wait
+// that gave up (set with atomicCAS so the first cause is kept).
+enum DeviceStatus : unsigned int {
+    kDevOk = 0,
+    kDevWaitTimeout = 1,
+};
+
+// The word lives in api.cu; kernels receive its device address as an argument
+// (one translation unit per kernel family, no relocatable device code).
+__device__ __forceinline__ void record_status(unsigned int* status, unsigned int code)
+{
+    if (status) atomicCAS(status, 0u, code);
+}
+
+// I/O element access: fp32 or bf16 storage, fp32 arithmetic.
+template <typename T> struct io;
+template <> struct io<float> {
+    static __device__ __forceinline__ float load(const float* p) { return __ldg(p); }
+    static __device__ __forceinline__ void store(float* p, float v) { *p = v; }
+};
+template <> struct io<__nv_bfloat16> {
+    static __device__ __forceinline__ float load(const __nv_bfloat16* p)
+    {
+        return __bfloat162float(__ldg(p));
+    }
+    static __device__ __forceinline__ void store(__nv_bfloat16* p, float v)
+    {
+        *p = __float2bfloat16_rn(v);
+    }
+};
+
+// Per-call context every launcher receives from api.cu.
+struct LaunchCtx {
+    cudaStream_t stream;
+    unsigned int* status;        // device status word
+    unsigned long long wait_limit;  // iterations of a bounded device wait
+    int num_sms;
+};
+
+}  // namespace ssd
+
+namespace ssd {
+
+// Arguments of one forward call as the launchers see them (pointers are device
+// pointers; x, Bm, Cm, y are in the I/O dtype named by `bf16`).
+struct FwdArgs {
+    const void* x;
+    const float* dt;
+    const float* A;
+    const void* Bm;
+    const void* Cm;
+    const float* D;         // may be null
+    const float* init;      // may be null
+    void* y;
+    float* final_state;     // may be null
+    int B, L, H, P, G, N, chunk;
+    bool bf16;
+};
+
+struct StepArgs {
+    const void* x;
+    const float* dt;
+    const float* A;
+    const void* Bm;
+    const void* Cm;
+    const float* D;
+    float* state;
+    void* y;
+    int B, H, P, G, N;
+    bool bf16;
+};
+
+// SIMT path (simt_forward.cu): any valid size, fp32 arithmetic.
+size_t simt_workspace_bytes(const FwdArgs& a);
+cudaError_t simt_forward(const FwdArgs& a, void* workspace, const LaunchCtx& ctx);
+
+// Decode step (step.cu).
+cudaError_t step_forward(const StepArgs& a, const LaunchCtx& ctx);
+
+}  // namespace ssd

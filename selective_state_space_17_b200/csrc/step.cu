@@ -1,0 +1,150 @@
+// step.cu — single-token decode step of the SSD layer.
+//
+// Per (b, h): a = exp(dt A_h); state <- a * state + dt * x B^T; y = state C + D x.
+// This is the recurrent route the pages recommend for generation ("Mamba-2",
+// docsaid.org, section "Computing with four tokens": the recurrent form keeps a
+// constant-size state and suits generation), with the discretisation of
+// "Mamba paper review" (youngju.dev), section 3.3.
+//
+// The step is bound by HBM: the fp32 state is read and written once (P*N*8
+// bytes per head) and everything else is small. One CTA of 8 warps per (b, h);
+// a warp owns whole state rows p and moves them with 128-bit accesses (lane l
+// holds n = 4l .. 4l+3 of each 128-column stripe), four rows in flight per
+// warp, and reduces y_p with shuffles.
+#include "common.cuh"
+
+namespace ssd {
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kRowsInFlight = 4;
+
+template <typename T>
+__device__ __forceinline__ float4 load4(const T* p);
+template <>
+__device__ __forceinline__ float4 load4<float>(const float* p)
+{
+    return __ldg(reinterpret_cast<const float4*>(p));
+}
+template <>
+__device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bfloat16* p)
+{
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+    float4 f;
+    f.x = __uint_as_float(u.x << 16);
+    f.y = __uint_as_float(u.x & 0xffff0000u);
+    f.z = __uint_as_float(u.y << 16);
+    f.w = __uint_as_float(u.y & 0xffff0000u);
+    return f;
+}
+
+__device__ __forceinline__ float warp_sum(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Vector path: N % 4 == 0 (every row starts 16-byte aligned).
+template <typename T>
+__global__ void __launch_bounds__(kWarps * 32)
+step_vec(StepArgs a)
+{
+    const int bh = blockIdx.x;
+    const int b = bh / a.H, h = bh % a.H, g = h / (a.H / a.G);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const float d = a.dt[bh];
+    const float decay = expf(d * a.A[h]);
+    const float Dh = a.D ? a.D[h] : 0.f;
+    const T* x = static_cast<const T*>(a.x) + (size_t)bh * a.P;
+    const T* Bv = static_cast<const T*>(a.Bm) + ((size_t)b * a.G + g) * a.N;
+    const T* Cv = static_cast<const T*>(a.Cm) + ((size_t)b * a.G + g) * a.N;
+    T* y = static_cast<T*>(a.y) + (size_t)bh * a.P;
+    float* st = a.state + (size_t)bh * a.P * a.N;
+
+    for (int p0 = warp * kRowsInFlight; p0 < a.P; p0 += kWarps * kRowsInFlight) {
+        float acc[kRowsInFlight];
+        float u[kRowsInFlight];
+#pragma unroll
+        for (int r = 0; r < kRowsInFlight; ++r) {
+            acc[r] = 0.f;
+            u[r] = (p0 + r < a.P) ? d * io<T>::load(x + p0 + r) : 0.f;
+        }
+        for (int n = lane * 4; n < a.N; n += 128) {
+            const float4 bq = load4<T>(Bv + n);
+            const float4 cq = load4<T>(Cv + n);
+            float4 hv[kRowsInFlight];
+#pragma unroll
+            for (int r = 0; r < kRowsInFlight; ++r)
+                if (p0 + r < a.P)
+                    hv[r] = __ldcs(reinterpret_cast<const float4*>(st + (size_t)(p0 + r) * a.N + n));
+#pragma unroll
+            for (int r = 0; r < kRowsInFlight; ++r) {
+                if (p0 + r >= a.P) continue;
+                float4 v = hv[r];
+                v.x = decay * v.x + u[r] * bq.x;
+                v.y = decay * v.y + u[r] * bq.y;
+                v.z = decay * v.z + u[r] * bq.z;
+                v.w = decay * v.w + u[r] * bq.w;
+                acc[r] += v.x * cq.x + v.y * cq.y + v.z * cq.z + v.w * cq.w;
+                __stcs(reinterpret_cast<float4*>(st + (size_t)(p0 + r) * a.N + n), v);
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < kRowsInFlight; ++r) {
+            const float s = warp_sum(acc[r]);
+            if (lane == 0 && p0 + r < a.P)
+                io<T>::store(y + p0 + r, s + Dh * io<T>::load(x + p0 + r));
+        }
+    }
+}
+
+// Scalar path: any N.
+template <typename T>
+__global__ void __launch_bounds__(kWarps * 32)
+step_scalar(StepArgs a)
+{
+    const int bh = blockIdx.x;
+    const int b = bh / a.H, h = bh % a.H, g = h / (a.H / a.G);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const float d = a.dt[bh];
+    const float decay = expf(d * a.A[h]);
+    const float Dh = a.D ? a.D[h] : 0.f;
+    const T* x = static_cast<const T*>(a.x) + (size_t)bh * a.P;
+    const T* Bv = static_cast<const T*>(a.Bm) + ((size_t)b * a.G + g) * a.N;
+    const T* Cv = static_cast<const T*>(a.Cm) + ((size_t)b * a.G + g) * a.N;
+    T* y = static_cast<T*>(a.y) + (size_t)bh * a.P;
+    float* st = a.state + (size_t)bh * a.P * a.N;
+    for (int p = warp; p < a.P; p += kWarps) {
+        const float u = d * io<T>::load(x + p);
+        float acc = 0.f;
+        for (int n = lane; n < a.N; n += 32) {
+            float* hv = st + (size_t)p * a.N + n;
+            const float v = decay * *hv + u * io<T>::load(Bv + n);
+            *hv = v;
+            acc += v * io<T>::load(Cv + n);
+        }
+        acc = warp_sum(acc);
+        if (lane == 0) io<T>::store(y + p, acc + Dh * io<T>::load(x + p));
+    }
+}
+
+template <typename T>
+cudaError_t run(const StepArgs& a, const LaunchCtx& ctx)
+{
+    const int grid = a.B * a.H;
+    if (a.N % 4 == 0)
+        step_vec<T><<<grid, kWarps * 32, 0, ctx.stream>>>(a);
+    else
+        step_scalar<T><<<grid, kWarps * 32, 0, ctx.stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t step_forward(const StepArgs& a, const LaunchCtx& ctx)
+{
+    return a.bf16 ? run<__nv_bfloat16>(a, ctx) : run<float>(a, ctx);
+}
+
+}  // namespace ssd

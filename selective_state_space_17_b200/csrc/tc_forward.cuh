@@ -1,0 +1,13 @@
+// tc_forward.cuh — launcher interface of the tensor-core (tcgen05) forward path.
+#pragma once
+#include "common.cuh"
+
+namespace ssd {
+
+// True when the bf16 tensor-core path handles these sizes.
+bool tc_supported(const FwdArgs& a);
+size_t tc_workspace_bytes(const FwdArgs& a);
+cudaError_t tc_forward(const FwdArgs& a, void* workspace, const LaunchCtx& ctx);
+int tc_kernel_count(const FwdArgs& a);
+
+}  // namespace ssd

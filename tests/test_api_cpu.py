@@ -1,0 +1,122 @@
+"""Host-side checks of the C ABI that need no GPU: the library builds and
+loads, exports every entry point ``include/ssd.h`` declares, sizes its
+workspace, and rejects bad arguments before anything reaches the device.
+Every call here fails validation before the first CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from selective_state_space_17_b200 import build
+    build.build()
+    from selective_state_space_17_b200 import ssd
+    return ssd.lib
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(ssd_[a-z_0-9]+)\s*\(", text))
+    return names
+
+
+def test_library_exports_every_declared_entry_point(lib):
+    names = _declared()
+    assert {"ssd_forward", "ssd_step", "ssd_workspace_size", "ssd_poll_status"} <= names
+    for n in sorted(names):
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        s = lib.ssd_status_string(code).decode()
+        assert s.startswith("SSD_")
+    assert lib.ssd_status_string(99).decode() == "SSD_ERR_UNKNOWN"
+
+
+def test_workspace_size(lib):
+    assert lib.ssd_workspace_size(4, 4096, 80, 64, 1, 128, 256, 1) > 0
+    assert lib.ssd_workspace_size(1, 64, 2, 8, 1, 8, 16, 0) > 0
+    assert lib.ssd_workspace_size(1, 64, 3, 8, 2, 8, 16, 0) == 0   # H % G != 0
+    assert lib.ssd_workspace_size(1, 64, 2, 8, 1, 8, 0, 0) == 0    # chunk 0
+    assert lib.ssd_workspace_size(1, 64, 2, 512, 1, 8, 16, 0) == 0  # P too large
+    assert lib.ssd_workspace_size(1, 64, 2, 8, 1, 8, 16, 7) == 0   # bad dtype
+    a = lib.ssd_workspace_size(1, 4096, 2, 64, 1, 64, 128, 1)
+    b = lib.ssd_workspace_size(1, 8192, 2, 64, 1, 64, 128, 1)
+    assert b >= a
+
+
+P16 = [0x10000 * (i + 1) for i in range(10)]  # aligned, never dereferenced
+
+
+def _fwd(lib, ptrs, dims, ws_bytes=1 << 40):
+    x, dt, A, Bm, Cm, D, init, y, fs, ws = ptrs
+    return lib.ssd_forward(x, dt, A, Bm, Cm, D, init, y, fs, *dims, ws, ws_bytes, None)
+
+
+def test_forward_rejects_bad_arguments_before_launch(lib):
+    dims = (1, 64, 2, 8, 1, 8, 16, 0)
+    bad_dims = [(1, 64, 3, 8, 2, 8, 16, 0), (-1, 64, 2, 8, 1, 8, 16, 0),
+                (1, -5, 2, 8, 1, 8, 16, 0), (1, 64, 0, 8, 1, 8, 16, 0),
+                (1, 64, 2, 8, 1, 8, 0, 0), (1, 64, 2, 8, 1, 8, 16, 5)]
+    for d in bad_dims:
+        assert _fwd(lib, P16, d) == 1, d
+    for d in [(1, 64, 2, 300, 1, 8, 16, 0), (1, 64, 2, 8, 1, 300, 16, 0),
+              (1, 64, 2, 8, 1, 8, 512, 0)]:
+        assert _fwd(lib, P16, d) == 2, d
+    for k in (0, 1, 2, 3, 4, 7):  # required pointers
+        ptrs = list(P16)
+        ptrs[k] = None
+        assert _fwd(lib, ptrs, dims) == 1, k
+    for k in range(10):  # every pointer, optional ones included, must be aligned
+        ptrs = list(P16)
+        ptrs[k] += 4
+        assert _fwd(lib, ptrs, dims) == 3, k
+    ptrs = list(P16)
+    ptrs[9] = None
+    assert _fwd(lib, ptrs, dims) == 6
+    assert _fwd(lib, P16, dims, ws_bytes=16) == 6
+
+
+def test_step_rejects_bad_arguments_before_launch(lib):
+    ok = P16[:8]
+    assert lib.ssd_step(*ok, 2, 3, 8, 2, 8, 0, None) == 1   # H % G
+    assert lib.ssd_step(*ok, 2, 2, 8, 1, 8, 9, None) == 1   # dtype
+    assert lib.ssd_step(*ok, 2, 2, 999, 1, 8, 0, None) == 2
+    for k in (0, 1, 2, 3, 4, 6, 7):
+        ptrs = list(ok)
+        ptrs[k] = None
+        assert lib.ssd_step(*ptrs, 2, 2, 8, 1, 8, 0, None) == 1, k
+    ptrs = list(ok)
+    ptrs[6] += 8
+    assert lib.ssd_step(*ptrs, 2, 2, 8, 1, 8, 0, None) == 3
+
+
+def test_host_entry_rejects_small_buffer(lib):
+    need = lib.ssd_forward_host_buffer_size(1, 64, 2, 8, 1, 8, 16, 0)
+    assert need > lib.ssd_workspace_size(1, 64, 2, 8, 1, 8, 16, 0)
+    rc = lib.ssd_forward_host(*P16[:9], 1, 64, 2, 8, 1, 8, 16, 0, P16[9], need - 1, None)
+    assert rc == 6
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    """The Python binding has no fallback: a missing library is an ImportError."""
+    import subprocess
+    import sys
+    code = ("import os, sys, importlib.util; "
+            "spec = importlib.util.spec_from_file_location('ssd_copy', sys.argv[1]); "
+            "m = importlib.util.module_from_spec(spec); spec.loader.exec_module(m)")
+    src = os.path.join(ROOT, "selective_state_space_17_b200", "ssd.py")
+    copy = tmp_path / "ssd.py"
+    copy.write_text(open(src).read())
+    r = subprocess.run([sys.executable, "-c", code, str(copy)], capture_output=True, text=True)
+    assert r.returncode != 0 and "ImportError" in r.stderr and "no CPU" in r.stderr
