@@ -139,6 +139,13 @@ ssd_status ssd_poll_status(ssd_stream_t stream);
  * up at once, which exercises the timeout path without hanging anything. */
 void ssd_set_wait_limit(uint64_t iterations);
 
+/* Test hook: when `skip_publish` is nonzero, forward calls on the tensor-core
+ * path never publish tile end states, so every look-back wait runs into the
+ * iteration limit and the call reports SSD_ERR_TIMEOUT through
+ * ssd_poll_status(). Results of such calls are garbage. 0 restores normal
+ * operation. */
+void ssd_set_fault_injection(int skip_publish);
+
 #ifdef __cplusplus
 }
 #endif

@@ -15,7 +15,7 @@ __device__ unsigned int g_device_status;
 
 namespace {
 
-constexpr unsigned long long kDefaultWaitLimit = 1ull << 26;  // ~seconds of polling
+constexpr unsigned long long kDefaultWaitLimit = 1ull << 23;  // ~seconds of polling
 constexpr int kMaxDevices = 64;
 
 unsigned long long g_wait_limit = kDefaultWaitLimit;
@@ -269,6 +269,8 @@ ssd_status ssd_poll_status(ssd_stream_t stream)
     }
     return SSD_OK;
 }
+
+void ssd_set_fault_injection(int skip_publish) { tc_set_skip_publish(skip_publish); }
 
 void ssd_set_wait_limit(uint64_t iterations)
 {

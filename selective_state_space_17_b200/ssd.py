@@ -43,6 +43,8 @@ lib.ssd_poll_status.argtypes = [_vp]
 lib.ssd_poll_status.restype = _i
 lib.ssd_forward_kernel_count.argtypes = [_i] * 8
 lib.ssd_forward_kernel_count.restype = _i
+lib.ssd_set_fault_injection.argtypes = [_i]
+lib.ssd_set_fault_injection.restype = None
 lib.ssd_set_wait_limit.argtypes = [ctypes.c_uint64]
 lib.ssd_set_wait_limit.restype = None
 
@@ -204,4 +206,10 @@ def poll_status(stream=None) -> None:
 
 
 def set_wait_limit(iterations: int) -> None:
+    """Iteration limit of device-side look-back waits (0 restores the default)."""
     lib.ssd_set_wait_limit(int(iterations))
+
+
+def set_fault_injection(skip_publish: bool) -> None:
+    """Test hook: tiles stop publishing end states (see include/ssd.h)."""
+    lib.ssd_set_fault_injection(1 if skip_publish else 0)
