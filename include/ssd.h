@@ -99,6 +99,27 @@ ssd_status ssd_forward(const void* x, const float* dt, const float* A, const voi
                        ssd_stream_t stream);
 
 /*
+ * ssd_forward_noalloc — the forward pass for callers that cannot allocate
+ * device memory. The pages describe no such entry point; it is a convenience
+ * of this library. It takes the same arguments as ssd_forward without the
+ * workspace: its scratch (look-back control words and the per-head state
+ * ring, 256 + 4*B*H rounded to 256 + 2*B*H*P*N*4 bytes) lives in a fixed
+ * 24 MiB device array inside the library, which every GPU that loads the
+ * library holds until the process exits. Only the tensor-core sizes are
+ * handled (bf16, P == 64, N == 128, chunk 128 or 256, B*L > 0); other sizes
+ * return SSD_ERR_UNSUPPORTED, and sizes whose scratch exceeds the array
+ * (B*H > 383 at N == 128) return SSD_ERR_WORKSPACE before anything is
+ * enqueued. The call allocates nothing. The first call on each device looks
+ * up the array's device address (make it before any stream capture). All
+ * calls on a device share the array: calls that may overlap on the GPU race
+ * and must not be issued concurrently; calls ordered on one stream are safe.
+ */
+ssd_status ssd_forward_noalloc(const void* x, const float* dt, const float* A, const void* Bm,
+                               const void* Cm, const float* D, const float* initial_state,
+                               void* y, float* final_state, int B, int L, int H, int P, int G,
+                               int N, int chunk, ssd_dtype dtype, ssd_stream_t stream);
+
+/*
  * ssd_forward_host — the same forward pass on HOST buffers (pinned memory
  * gives asynchronous copies). Copies the inputs into `device_buffer`, runs
  * ssd_forward on `stream`, copies y (and final_state if non-NULL) back, and

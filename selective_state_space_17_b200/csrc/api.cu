@@ -92,6 +92,9 @@ ssd_status empty_forward(const FwdArgs& a, cudaStream_t stream)
 }
 
 }  // namespace
+
+ssd_status acquire_launch_ctx(cudaStream_t stream, LaunchCtx* ctx) { return make_ctx(stream, ctx); }
+
 }  // namespace ssd
 
 using namespace ssd;

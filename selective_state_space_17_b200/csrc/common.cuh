@@ -85,6 +85,10 @@ struct StepArgs {
 size_t simt_workspace_bytes(const FwdArgs& a);
 cudaError_t simt_forward(const FwdArgs& a, void* workspace, const LaunchCtx& ctx);
 
+// Device status word, stream and limits for a launch on the current device
+// (api.cu).
+ssd_status acquire_launch_ctx(cudaStream_t stream, LaunchCtx* ctx);
+
 // Decode step (step.cu).
 cudaError_t step_forward(const StepArgs& a, const LaunchCtx& ctx);
 

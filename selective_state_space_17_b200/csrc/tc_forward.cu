@@ -537,3 +537,86 @@ cudaError_t tc_forward(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)
 }
 
 }  // namespace ssd
+
+// ---------------------------------------------------------------------------
+// Allocation-free forward pass.
+//
+// Some callers cannot allocate device memory: code that runs where an
+// allocation is not allowed or would be unsafe (for instance inside a
+// framework callback that must not call cudaMalloc, on a memory pool that is
+// already full, or in an embedded host that owns every byte of device memory)
+// and callers that have no convenient place to keep a workspace alive between
+// calls. For them, ssd_forward_noalloc runs the tensor-core forward with its
+// scratch (look-back control words and the per-head state ring) in the fixed
+// device array below instead of a caller-provided workspace. The caller still
+// passes every input and output buffer.
+//
+// The array belongs to the library: each GPU that loads it holds the array
+// until the process exits. Every call on a device shares it and leaves its
+// contents behind, so calls that may overlap on the GPU (different streams,
+// or host threads without ordering) race and must not be issued; calls on one
+// stream are ordered and safe. Host code cannot use the array's name as a
+// device address, so the first call on each device looks its address up with
+// cudaGetSymbolAddress (make that first call before any stream capture).
+namespace ssd {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(24) << 20;  // 24 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoAllocMaxDevices];
+
+bool noalloc_aligned(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; }
+
+}  // namespace
+}  // namespace ssd
+
+extern "C" ssd_status ssd_forward_noalloc(const void* x, const float* dt, const float* A,
+                                          const void* Bm, const void* Cm, const float* D,
+                                          const float* initial_state, void* y,
+                                          float* final_state, int B, int L, int H, int P, int G,
+                                          int N, int chunk, ssd_dtype dtype, ssd_stream_t stream)
+{
+    using namespace ssd;
+    if (B < 0 || L < 0 || H < 1 || G < 1 || P < 1 || N < 1 || chunk < 1 || H % G != 0 ||
+        (dtype != SSD_F32 && dtype != SSD_BF16))
+        return SSD_ERR_INVALID_ARG;
+    if ((long long)B * L == 0) return SSD_ERR_UNSUPPORTED;  // nothing for the scratch to do
+    if (!x || !dt || !A || !Bm || !Cm || !y) return SSD_ERR_INVALID_ARG;
+    const void* ptrs[] = {x, dt, A, Bm, Cm, D, initial_state, y, final_state};
+    for (const void* q : ptrs)
+        if (q && !noalloc_aligned(q)) return SSD_ERR_MISALIGNED;
+    FwdArgs a;
+    a.x = x; a.dt = dt; a.A = A; a.Bm = Bm; a.Cm = Cm; a.D = D; a.init = initial_state;
+    a.y = y; a.final_state = final_state;
+    a.B = B; a.L = L; a.H = H; a.P = P; a.G = G; a.N = N; a.chunk = chunk;
+    a.bf16 = dtype == SSD_BF16;
+    if (!tc_supported(a)) return SSD_ERR_UNSUPPORTED;  // tensor-core sizes only
+    const WsLayout w = ws_layout(a);
+    if (w.total > kNoAllocScratchBytes) return SSD_ERR_WORKSPACE;  // scratch would not fit
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices)
+        return SSD_ERR_CUDA;
+    void* scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_noalloc_mu);
+        if (!g_noalloc_ptr[dev]) {
+            void* addr = nullptr;
+            if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || !addr)
+                return SSD_ERR_CUDA;
+            g_noalloc_ptr[dev] = addr;
+        }
+        scratch = g_noalloc_ptr[dev];
+    }
+    LaunchCtx ctx;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const ssd_status st = acquire_launch_ctx(s, &ctx);
+    if (st != SSD_OK) return st;
+    // the ticket, done counter and look-back flags must start at zero
+    if (cudaMemsetAsync(scratch, 0, w.ring, s) != cudaSuccess) return SSD_ERR_CUDA;
+    const cudaError_t e = tc_forward(a, scratch, ctx);
+    return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
