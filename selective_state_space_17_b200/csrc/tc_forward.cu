@@ -1,32 +1,51 @@
 // tc_forward.cu — tensor-core (tcgen05) forward path of the SSD layer.
 //
 // The chunked algorithm of "Mamba-2" (docsaid.org), section "Half of each
-// route": inside a tile the quadratic ("attention") form runs on the tensor
-// cores; across tiles only the end state is carried. Each CTA takes one work
-// item = one head of one batch row over one 128-token tile (item order is
-// tile-major, handed out by an atomic ticket so that an item's predecessor on
-// the same head always started earlier). Per item, with cs the tile-local
-// cumulative sum of dt * A (log2 units), everything on chip:
+// route": inside a 128-token tile the quadratic ("attention") form runs on the
+// tensor cores; across tiles only the end state is carried. Per tile, with cs
+// the tile-local cumulative sum of dt * A (log2 units):
 //
-//   1. TMA loads C, B (128 x N) and X (128 x 64) tiles (128-byte swizzle).
-//   2. MMA1:   S  = C B^T                  (128 x 128, K = N)       -> TMEM
-//      states: s  = B^T (w o X), w_j = exp(cs_end - cs_j) dt_j
-//                                          (N x 64, K = 128)        -> TMEM
-//   3. mask:   S~_ij = S_ij exp(cs_i - cs_j) dt_j for j <= i, else 0 (bf16, smem)
-//      MMA2:   Yd = S~ X                   (128 x 64, K = 128)      -> TMEM
-//   4. look-back: wait until the head's previous tile published h_prev
-//      (fp32, [P][N], in a two-slot ring of the workspace), then
-//      h = exp(cs_end) h_prev + s is published for the next tile (or written
-//      to final_state), and h_prev in bf16 feeds
-//      MMA3:   Ys = C h_prev^T              (128 x 64, K = N)       -> TMEM
-//   5. y_i = Yd_i + exp(cs_i) Ys_i + D x_i, stored as bf16.
+//   MMA1    S  = C B^T                                  (128 x 128, K = N)  TMEM
+//   states  s  = B^T (w o X),  w_j = exp(cs_end - cs_j) dt_j  (N x 64, K = 128) TMEM
+//   mask    S~_ij = S_ij exp(cs_i - cs_j) dt_j (j <= i), plus D_h on the diagonal,
+//           in registers, written as bf16 over the tile's B in shared memory
+//   MMA2    Yd = S~ X                                   (128 x 64, K = 128) TMEM
+//   MMA3    Ys = C h_prev^T                             (128 x 64, K = N)   TMEM
+//   output  y_i = Yd_i + exp(cs_i) Ys_i (bf16, round to nearest even)
+//   state   h = exp(cs_end) h_prev + s
 //
 // The masked product is the structured masked attention of "Mamba-2 SSD note"
 // (0h-n0.github.io), section "SSD layer: equivalence under the scalar
-// constraint" (C as queries, B as keys, X as values); the tile states are the
-// low-rank representation of the blocks below the diagonal ("Mamba-2",
-// section "Half of each route"); carrying h across tiles is the composition of
-// affine maps of "Selective SSM guide" (auturnal.com), eq. (3).
+// constraint" (C as queries, B as keys, X as values, D x folded in as the
+// diagonal D_h I); the tile states are the low-rank representation of the
+// blocks below the diagonal ("Mamba-2", section "Half of each route"); carrying
+// h is the composition of affine maps of "Selective SSM guide"
+// (auturnal.com), eq. (3). The mask's exponentials are factored per 32-column
+// block: for a block wholly left of row i with last column a,
+// exp(cs_i - cs_j) = exp(cs_i - cs_a) * exp(cs_a - cs_j), both factors <= 1,
+// so only the block on the diagonal needs one exponential per element.
+//
+// Schedule. Each (batch row, head) is a chain of tiles; chains are cut into
+// segments of `seg_len` tiles. A work item is one segment of one chain, and
+// items are numbered segment-major, so an item's predecessor (the previous
+// segment of the same chain) is numbered `chains` earlier. One persistent CTA
+// per SM takes items blockIdx.x, blockIdx.x + gridDim.x, ... and walks each
+// item's tiles in order with the state h kept in registers; only at a segment
+// boundary does h travel through the workspace (a two-slot fp32 ring per
+// chain, published with a release flag and read after a bounded acquire poll).
+//
+// Warp roles inside the CTA (384 threads), linked by full/empty mbarrier rings
+// whose waits sleep rather than spin:
+//   warp 0        TMA producer: C, B (2 stages), X (3 stages), L2 prefetch of
+//                 the X tiles further ahead
+//   warp 1        MMA issuer, one tile of lag: MMA1 and states of tile k are
+//                 issued before MMA2 and MMA3 of tile k-1, so the tensor core
+//                 works on tile k while tile k-1 is being masked (S is double
+//                 buffered in TMEM)
+//   warps 2-3     tile prologue: cumsum, column factors, w o X
+//   warps 4-7     mask S -> S~
+//   warps 8-11    h_prev -> bf16 operand, state update, epilogue, look-back
+//                 and segment publication
 //
 // A chunk of 256 tokens is evaluated as two 128-token tiles: its quadratic
 // form split into 2 x 2 blocks, the diagonal blocks computed directly and the
@@ -47,18 +66,35 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kT = 128;        // tokens per tile
-constexpr int kP = 64;         // head dim on this path
-constexpr int kThreads = 128;  // 4 warps: thread i <-> tile row / TMEM lane i
+constexpr int kT = 128;   // tokens per tile
+constexpr int kP = 64;    // head dim on this path
+constexpr int kN = 128;   // state dim on this path
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr uint64_t kMbarLimit = 1ull << 22;  // hardware-completion waits (~seconds)
+constexpr uint64_t kMbarLimit = 1ull << 22;  // polls; each wait is also capped at ~2 s
 
-// TMEM columns (fp32 accumulators, 128 lanes each)
-constexpr uint32_t kColS = 0;      // S: 128 columns
-constexpr uint32_t kColState = 128;  // s: 64 columns per 128 rows of N
-constexpr uint32_t kColYd = 256;   // Yd: 64
-constexpr uint32_t kColYs = 320;   // Ys: 64
+constexpr int kThreads = 384;
+constexpr int kWarpProducer = 0;
+constexpr int kWarpMma = 1;
+constexpr int kWarpPrep0 = 2;  // warps 2..3
+constexpr int kWarpAlloc = 2;
+constexpr int kWgMask0 = 4;    // warps 4..7
+constexpr int kWgOut0 = 8;     // warps 8..11
+constexpr int kBarPrep = 1;    // named barrier ids
+constexpr int kBarOut = 2;
+
+constexpr int kCbStages = 2;
+constexpr int kXStages = 3;
+constexpr int kCsStages = 4;
+constexpr int kPrefetchAhead = 4;
+
+// TMEM columns (fp32, 128 lanes)
+constexpr uint32_t kColS = 0;     // 2 x 128: S, then S~ (bf16, cols 0-63) and Ys (cols 64-127)
+constexpr uint32_t kColSt = 256;  // 2 x 64: tile states, lanes = n
+constexpr uint32_t kColY = 384;   // 2 x 64: Yd
 constexpr uint32_t kTmemCols = 512;
+
+constexpr uint32_t kTileBytesCB = kT * kN * 2;  // one C or B tile: 32 KB
+constexpr uint32_t kTileBytesX = kT * kP * 2;   // one X tile: 16 KB
 
 struct TcParams {
     const float* dt;
@@ -67,34 +103,97 @@ struct TcParams {
     const float* init;
     __nv_bfloat16* y;
     float* final_state;
-    unsigned int* ctrl;   // [0] ticket, [1] CTAs done
-    unsigned int* flags;  // per (b, h): number of tiles published
-    float* ring;          // per (b, h): 2 x [P][N] fp32
+    unsigned int* ctrl;   // [1] CTAs done
+    unsigned int* flags;  // per chain: number of segments published
+    float* ring;          // per chain: 2 slots of [N][P] fp32
     unsigned int* status;
     unsigned long long wait_limit;
-    int B, L, H, G, N, ntiles, total, chains;
-    int skip_publish;  // fault-injection hook: never publish states
+    int B, L, H, G;
+    int ntiles;   // tiles per chain
+    int chains;   // B * H
+    int seg_len;  // tiles per segment
+    int nseg;     // segments per chain
+    int items;    // chains * nseg
+    int skip_publish;
 };
 
-template <int N>
+// Per-tile prologue record (one per cumsum stage).
+struct TileRec {
+    float cs[kT];    // cumulative dt * A, log2 units
+    float dt[kT];
+    float colf[kT];  // exp2(cs[j | 31] - cs[j]) * dt[j]
+    float w[kT];     // exp2(cs[kT - 1] - cs[j]) * dt[j]
+    float Dh;
+    float pad[31];
+};
+
+// Shared memory (offsets from a 1024-aligned base).
 struct Smem {
-    static constexpr uint32_t kC = 0;
-    static constexpr uint32_t kB = kC + N * 256;      // N/64 regions of 16 KB
-    static constexpr uint32_t kX = kB + N * 256;
-    static constexpr uint32_t kXt = kX + 16384;
-    static constexpr uint32_t kSt = kXt + 16384;       // 2 regions of 16 KB
-    static constexpr uint32_t kHs = kSt + 32768;       // N/64 regions of 8 KB
-    static constexpr uint32_t kMisc = kHs + N * 128;
-    static constexpr uint32_t kCs = kMisc;             // 128 floats
-    static constexpr uint32_t kDt = kCs + 512;
-    static constexpr uint32_t kW = kDt + 512;
-    static constexpr uint32_t kRed = kW + 512;         // 8 floats
-    static constexpr uint32_t kBars = kRed + 64;       // 4 mbarriers
-    static constexpr uint32_t kTmemPtr = kBars + 32;
-    static constexpr uint32_t kItem = kTmemPtr + 4;
-    static constexpr uint32_t kFlag = kItem + 4;
-    static constexpr uint32_t kEnd = kFlag + 8;
-    static constexpr uint32_t kBytes = kEnd + 1024;    // + alignment slack
+    static constexpr uint32_t kC = 0;                                   // 2 x 32 KB
+    static constexpr uint32_t kB = kC + kCbStages * kTileBytesCB;       // 2 x 32 KB (B, then S~)
+    static constexpr uint32_t kX = kB + kCbStages * kTileBytesCB;       // 3 x 16 KB
+    static constexpr uint32_t kXt = kX + kXStages * kTileBytesX;        // 16 KB
+    static constexpr uint32_t kHs = kXt + kTileBytesX;                  // N x 64 bf16
+    static constexpr uint32_t kRec = kHs + kN * kP * 2;                 // 4 x TileRec
+    static constexpr uint32_t kRed = kRec + kCsStages * sizeof(TileRec);  // 8 floats
+    static constexpr uint32_t kBars = kRed + 32;
+    static constexpr int kNumBars = 40;
+    static constexpr uint32_t kTmemPtr = kBars + kNumBars * 8;
+    static constexpr uint32_t kAbort = kTmemPtr + 4;
+    static constexpr uint32_t kEnd = kAbort + 4;
+    static constexpr uint32_t kBytes = kEnd + 1024;  // alignment slack
+};
+static_assert(Smem::kBytes <= 227 * 1024, "shared memory budget");
+
+// mbarrier indices
+enum Bar : int {
+    kFullCB = 0,      // 2
+    kEmptyCB = 2,     // 2: the commit after MMA3 frees C and B of the stage
+    kFullX = 4,       // 3
+    kEmptyX = 7,      // 3
+    kFullXt = 10,
+    kEmptyXt = 11,
+    kFullRec = 12,    // 4
+    kEmptyRec = 16,   // 4 (five arrivals: the four mask warps and the output warpgroup)
+    kFullS = 20,      // 2: MMA1 done (S readable)
+    kFullSt = 22,     // 2: S~ written over S in TMEM (one arrival per mask warp)
+    kFullStates = 24, // 2
+    kEmptyStates = 26,// 2
+    kFullHs = 28,     // h_prev operand written
+    kEmptyHs = 29,
+    kFullY = 30,      // 2
+    kEmptyY = 32,     // 2
+    kDrain = 34,
+};
+
+// Position in this CTA's sequence of tiles (identical in every role).
+struct Seq {
+    int item, tile, tile_end, seg, chain, b, h;
+    bool valid;
+
+    __device__ void setup(const TcParams& p)
+    {
+        valid = item < p.items;
+        if (!valid) return;
+        seg = item / p.chains;
+        chain = item - seg * p.chains;
+        b = chain / p.H;
+        h = chain - b * p.H;
+        tile = seg * p.seg_len;
+        tile_end = min(tile + p.seg_len, p.ntiles);
+    }
+    __device__ void begin(const TcParams& p)
+    {
+        item = blockIdx.x;
+        setup(p);
+    }
+    __device__ void next(const TcParams& p)
+    {
+        if (++tile >= tile_end) {
+            item += gridDim.x;
+            setup(p);
+        }
+    }
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
@@ -108,41 +207,59 @@ __device__ __forceinline__ float2 unpack_bf16x2(uint32_t u)
     return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
 }
 
-template <int N>
+__device__ __forceinline__ uint4 scale_bf16x8(uint4 q, float f)
+{
+    uint32_t* u = reinterpret_cast<uint32_t*>(&q);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 v = unpack_bf16x2(u[e]);
+        u[e] = pack_bf16x2(v.x * f, v.y * f);
+    }
+    return q;
+}
+
+// Bounded wait that turns a give-up into the CTA's abort mode: from then on
+// waits return at once, every role runs to the end of its loop on whatever is
+// in its buffers, and the device status word reports the timeout.
+__device__ __forceinline__ void wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                        unsigned int* status)
+{
+    if (*abort_flag) return;
+    if (!mbar_wait(bar, parity, kMbarLimit)) {
+        record_status(status, kDevWaitTimeout);
+        *abort_flag = 1;
+    }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmC, TcParams p)
 {
-    using S = Smem<N>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-    float* s_cs = reinterpret_cast<float*>(sm + S::kCs);
-    float* s_dt = reinterpret_cast<float*>(sm + S::kDt);
-    float* s_w = reinterpret_cast<float*>(sm + S::kW);
-    float* s_red = reinterpret_cast<float*>(sm + S::kRed);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + S::kBars);
-    uint64_t* bar_tma = bars + 0;
-    uint64_t* bar_mma1 = bars + 1;
-    uint64_t* bar_mma2 = bars + 2;
-    uint64_t* bar_mma3 = bars + 3;
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + S::kTmemPtr);
-    int* s_item = reinterpret_cast<int*>(sm + S::kItem);
-    int* s_flag = reinterpret_cast<int*>(sm + S::kFlag);
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte alignment for the swizzle atoms, by offsetting the shared array
+    // itself so that every access below stays in the shared address space
+    uint8_t* sm = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Smem::kBars);
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + Smem::kTmemPtr);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Smem::kAbort);
+    TileRec* recs = reinterpret_cast<TileRec*>(sm + Smem::kRec);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
+    const int lane = tid & 31;
 
     if (tid == 0) {
         prefetch_tensormap(&tmX);
         prefetch_tensormap(&tmB);
         prefetch_tensormap(&tmC);
-        for (int i = 0; i < 4; ++i) mbar_init(bars + i, 1);
+        for (int i = 0; i < Smem::kNumBars; ++i)
+            mbar_init(bars + i, (i >= kEmptyRec && i < kEmptyRec + kCsStages) ? 5u
+                                : (i >= kFullSt && i < kFullSt + 2)          ? 4u
+                                                                             : 1u);
         mbar_fence_init();
-        *s_item = static_cast<int>(atomicAdd(p.ctrl, 1u));
-        s_flag[0] = 0;  // set if a bounded wait gave up
+        *abort_flag = 0;
     }
-    if (warp == 0) {
+    if (warp == kWarpAlloc) {
         tmem_alloc(s_tmem, kTmemCols);
         tmem_relinquish();
     }
@@ -150,275 +267,445 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *s_tmem;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
 
-    const int item = *s_item;
-    const int tile = item / (p.B * p.H);
-    const int chain = item - tile * (p.B * p.H);
-    const int b = chain / p.H;
-    const int h = chain - b * p.H;
-    const int g = h / (p.H / p.G);
-    const int t0 = tile * kT;
-    const int rows = min(kT, p.L - t0);
-
-    // ---- 1. TMA loads
-    if (tid == 0) {
-        mbar_arrive_expect_tx(bar_tma, 2 * N * 256 + 16384);
+    if (warp == kWarpProducer) {
+        // ------------------------------------------------------------- producer
+        if (lane == 0) {
+            Seq s, pf;
+            s.begin(p);
+            pf.begin(p);
+            for (int d = 0; d < kPrefetchAhead && pf.valid; ++d) pf.next(p);
+            // X runs one tile ahead of C and B: its stage frees earlier
+            Seq sx = s;
+            auto load_x = [&](int kx) {
+                const int xs = kx % kXStages;
+                wait_bar(bars + kEmptyX + xs, ((kx / kXStages) & 1) ^ 1, abort_flag, p.status);
+                mbar_arrive_expect_tx(bars + kFullX + xs, kTileBytesX);
+                tma_load_4d(sm + Smem::kX + xs * kTileBytesX, &tmX, 0, sx.h, sx.tile * kT, sx.b,
+                            bars + kFullX + xs);
+                sx.next(p);
+            };
+            int kx = 0;
+            if (sx.valid) load_x(kx++);
+            int k = 0;
+            for (; s.valid; ++k, s.next(p)) {
+                if (pf.valid) {
+                    tma_prefetch_l2_4d(&tmX, 0, pf.h, pf.tile * kT, pf.b);
+                    pf.next(p);
+                }
+                const int g = s.h / (p.H / p.G);
+                const int t0 = s.tile * kT;
+                const int cb = k % kCbStages;
+                wait_bar(bars + kEmptyCB + cb, ((k / kCbStages) & 1) ^ 1, abort_flag, p.status);
+                mbar_arrive_expect_tx(bars + kFullCB + cb, 2 * kTileBytesCB);
 #pragma unroll
-        for (int k = 0; k < N / 64; ++k) {
-            tma_load_4d(sm + S::kC + k * 16384, &tmC, k * 64, g, t0, b, bar_tma);
-            tma_load_4d(sm + S::kB + k * 16384, &tmB, k * 64, g, t0, b, bar_tma);
-        }
-        tma_load_4d(sm + S::kX, &tmX, 0, h, t0, b, bar_tma);
-    }
-
-    // ---- tile-local cumulative sum of dt * A (log2 units)
-    const float Ah = p.A[h] * kLog2e;
-    const float dti = tid < rows ? p.dt[(static_cast<size_t>(b) * p.L + t0 + tid) * p.H + h] : 0.f;
-    float v = dti * Ah;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const float u = __shfl_up_sync(0xffffffffu, v, o);
-        if ((tid & 31) >= o) v += u;
-    }
-    if ((tid & 31) == 31) s_red[warp] = v;
-    __syncthreads();
-    for (int w = 0; w < warp; ++w) v += s_red[w];
-    s_cs[tid] = v;
-    s_dt[tid] = dti;
-    __syncthreads();
-    const float cs_end = s_cs[kT - 1];
-    const float cs_i = v;
-    s_w[tid] = exp2f(cs_end - cs_i) * dti;
-    __syncthreads();
-
-    // ---- wait for the tiles
-    if (!mbar_wait(bar_tma, 0, kMbarLimit)) {
-        record_status(p.status, kDevWaitTimeout);
-        s_flag[0] = 1;
-    }
-
-    // ---- X~ = w o X (row j of the swizzled tile is the 128 bytes at j * 128)
-    {
-        const uint4* src = reinterpret_cast<const uint4*>(sm + S::kX);
-        uint4* dst = reinterpret_cast<uint4*>(sm + S::kXt);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const int chunk = tid + k * kThreads;
-            const float wj = s_w[chunk >> 3];
-            uint4 q = src[chunk];
-            uint32_t* u = reinterpret_cast<uint32_t*>(&q);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = unpack_bf16x2(u[e]);
-                u[e] = pack_bf16x2(f.x * wj, f.y * wj);
+                for (int q = 0; q < kN / 64; ++q) {
+                    tma_load_4d(sm + Smem::kC + cb * kTileBytesCB + q * 16384, &tmC, q * 64, g, t0,
+                                s.b, bars + kFullCB + cb);
+                    tma_load_4d(sm + Smem::kB + cb * kTileBytesCB + q * 16384, &tmB, q * 64, g, t0,
+                                s.b, bars + kFullCB + cb);
+                }
+                if (sx.valid) load_x(kx++);
             }
-            dst[chunk] = q;
+            // drain: every load issued has landed before the CTA can exit
+            for (int j = max(0, k - kCbStages); j < k; ++j)
+                mbar_wait(bars + kFullCB + j % kCbStages, (j / kCbStages) & 1, kMbarLimit);
+            for (int j = max(0, kx - kXStages); j < kx; ++j)
+                mbar_wait(bars + kFullX + j % kXStages, (j / kXStages) & 1, kMbarLimit);
         }
-    }
-    fence_async_shared();
-    tc_fence_before_sync();
-    __syncthreads();
-
-    // ---- 2. MMA1 (S = C B^T) and the tile states (s = B^T X~)
-    if (tid == 0) {
-        tc_fence_after_sync();
-        const uint32_t c_base = smem_addr(sm + S::kC);
-        const uint32_t b_base = smem_addr(sm + S::kB);
-        const uint32_t xt_base = smem_addr(sm + S::kXt);
-        constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
+    } else if (warp == kWarpMma) {
+        // ----------------------------------------------- all MMAs, one tile of lag
+        // per iteration: MMA1 of tile k, MMA2 + MMA3 of tile k-1, states of tile k
+        if (lane == 0) {
+            constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
+            constexpr uint32_t id_st = idesc_bf16(128, kP, true, true);
+            constexpr uint32_t id_y2 = idesc_bf16(128, kP, false, true);
+            const uint32_t xt_base = smem_addr(sm + Smem::kXt);
+            const uint32_t hs_base = smem_addr(sm + Smem::kHs);
+            Seq s;
+            s.begin(p);
+            int k = 0;
+            bool prev = false;
+            for (;;) {
+                const bool cur = s.valid;
+                if (cur) {
+                    const int cb = k % kCbStages, sb = k & 1;
+                    const uint32_t c_base = smem_addr(sm + Smem::kC + cb * kTileBytesCB);
+                    const uint32_t b_base = smem_addr(sm + Smem::kB + cb * kTileBytesCB);
+                    wait_bar(bars + kFullCB + cb, (k / kCbStages) & 1, abort_flag, p.status);
+                    // S[sb] held S~ and Ys of tile k-2 until its epilogue read them
+                    if (k >= 2) wait_bar(bars + kEmptyY + sb, ((k - 2) >> 1) & 1, abort_flag, p.status);
+                    tc_fence_after_sync();
 #pragma unroll
-        for (int k = 0; k < N / 16; ++k) {
-            const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-            mma_bf16(tmem + kColS, sdesc_sw128(c_base + off, 16, 1024),
-                     sdesc_sw128(b_base + off, 16, 1024), id_s, k > 0);
-        }
-        constexpr uint32_t id_st = idesc_bf16(128, kP, true, true);
+                    for (int q = 0; q < kN / 16; ++q) {
+                        const uint32_t off = (q >> 2) * 16384 + (q & 3) * 32;
+                        mma_bf16(tmem + kColS + sb * 128, sdesc_sw128(c_base + off, 16, 1024),
+                                 sdesc_sw128(b_base + off, 16, 1024), id_s, q > 0);
+                    }
+                    mma_commit(bars + kFullS + sb);
+                }
+                if (prev) {
+                    const int j = k - 1;
+                    const int cb = j % kCbStages, xs = j % kXStages, sb = j & 1;
+                    const uint32_t c_base = smem_addr(sm + Smem::kC + cb * kTileBytesCB);
+                    const uint32_t x_base = smem_addr(sm + Smem::kX + xs * kTileBytesX);
+                    wait_bar(bars + kFullSt + sb, (j >> 1) & 1, abort_flag, p.status);
+                    wait_bar(bars + kEmptyY + sb, ((j >> 1) & 1) ^ 1, abort_flag, p.status);
+                    tc_fence_after_sync();
 #pragma unroll
-        for (int m = 0; m < N / 128; ++m) {
+                    for (int q = 0; q < kT / 16; ++q) {
+                        mma_bf16_tmem_a(tmem + kColY + sb * 64, tmem + kColS + sb * 128 + q * 8,
+                                        sdesc_sw128(x_base + q * 2048, 16384, 1024), id_y2, q > 0);
+                    }
+                    wait_bar(bars + kFullHs, j & 1, abort_flag, p.status);
+                    tc_fence_after_sync();
 #pragma unroll
-            for (int k = 0; k < kT / 16; ++k) {
-                mma_bf16(tmem + kColState + m * 64,
-                         sdesc_sw128(b_base + m * 32768 + k * 2048, 16384, 1024),
-                         sdesc_sw128(xt_base + k * 2048, 16384, 1024), id_st, k > 0);
+                    for (int q = 0; q < kN / 16; ++q) {
+                        mma_bf16(tmem + kColS + sb * 128 + 64,
+                                 sdesc_sw128(c_base + (q >> 2) * 16384 + (q & 3) * 32, 16, 1024),
+                                 sdesc_sw128(hs_base + q * 2048, 16384, 1024), id_y2, q > 0);
+                    }
+                    mma_commit(bars + kFullY + sb);
+                    mma_commit(bars + kEmptyHs);
+                    mma_commit(bars + kEmptyX + xs);
+                    mma_commit(bars + kEmptyCB + cb);
+                }
+                if (cur) {
+                    const int cb = k % kCbStages, sb = k & 1;
+                    const uint32_t b_base = smem_addr(sm + Smem::kB + cb * kTileBytesCB);
+                    wait_bar(bars + kEmptyStates + sb, ((k >> 1) & 1) ^ 1, abort_flag, p.status);
+                    wait_bar(bars + kFullXt, k & 1, abort_flag, p.status);
+                    tc_fence_after_sync();
+#pragma unroll
+                    for (int q = 0; q < kT / 16; ++q) {
+                        mma_bf16(tmem + kColSt + sb * 64,
+                                 sdesc_sw128(b_base + q * 2048, 16384, 1024),
+                                 sdesc_sw128(xt_base + q * 2048, 16384, 1024), id_st, q > 0);
+                    }
+                    mma_commit(bars + kEmptyXt);
+                    mma_commit(bars + kFullStates + sb);
+                }
+                if (!cur) break;
+                prev = true;
+                ++k;
+                s.next(p);
             }
+            mma_commit(bars + kDrain);
+            mbar_wait(bars + kDrain, 0, kMbarLimit);
         }
-        mma_commit(bar_mma1);
-    }
-    if (!mbar_wait(bar_mma1, 0, kMbarLimit)) {
-        record_status(p.status, kDevWaitTimeout);
-        s_flag[0] = 1;
-    }
-    tc_fence_after_sync();
+    } else if (warp >= kWarpPrep0 && warp < kWarpPrep0 + 2) {
+        // ------------------------------------- prologue: cumsum, factors, w o X
+        const int t = tid - kWarpPrep0 * 32;  // 0..63, tokens 2t and 2t + 1
+        const int wq = warp - kWarpPrep0;
+        float* red = reinterpret_cast<float*>(sm + Smem::kRed);
+        Seq s;
+        s.begin(p);
+        float2 dt_next = make_float2(0.f, 0.f);
+        float A_next = 0.f, D_next = 0.f;
+        auto fetch = [&](const Seq& q) {
+            const int rows = min(kT, p.L - q.tile * kT);
+            const size_t base = (static_cast<size_t>(q.b) * p.L + q.tile * kT) * p.H + q.h;
+            dt_next.x = 2 * t < rows ? p.dt[base + static_cast<size_t>(2 * t) * p.H] : 0.f;
+            dt_next.y = 2 * t + 1 < rows ? p.dt[base + static_cast<size_t>(2 * t + 1) * p.H] : 0.f;
+            A_next = p.A[q.h];
+            D_next = p.D ? p.D[q.h] : 0.f;
+        };
+        if (s.valid) fetch(s);
+        for (int k = 0; s.valid; ++k) {
+            const int c = k % kCsStages, xs = k % kXStages;
+            TileRec& r = recs[c];
+            const float2 dtv = dt_next;
+            const float Ah = A_next * kLog2e;
+            const float Dh = D_next;
+            s.next(p);
+            if (s.valid) fetch(s);
 
-    // ---- 3. mask S into S~ (bf16, K-major, two 64-column regions)
-    {
-        const int i = tid;
-        uint8_t* st = sm + S::kSt;
-#pragma unroll 1
-        for (int jb = 0; jb < 4; ++jb) {
-            float sv[32];
-            tmem_ld32(tmem + lane_off + kColS + jb * 32, sv);
-            tmem_wait_ld();
-            uint32_t packed[16];
+            wait_bar(bars + kEmptyRec + c, ((k / kCsStages) & 1) ^ 1, abort_flag, p.status);
+            const float a0 = dtv.x * Ah;
+            const float a1 = a0 + dtv.y * Ah;
+            float v = a1;
 #pragma unroll
-            for (int jj = 0; jj < 32; jj += 2) {
-                const int j0 = jb * 32 + jj, j1 = j0 + 1;
-                const float m0 = j0 <= i ? sv[jj] * exp2f(cs_i - s_cs[j0]) * s_dt[j0] : 0.f;
-                const float m1 = j1 <= i ? sv[jj + 1] * exp2f(cs_i - s_cs[j1]) * s_dt[j1] : 0.f;
-                packed[jj >> 1] = pack_bf16x2(m0, m1);
+            for (int o = 1; o < 32; o <<= 1) {
+                const float u = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += u;
             }
+            if (lane == 31) red[wq] = v;
+            named_bar_sync(kBarPrep, 64);
+            const float excl = v - a1 + (wq == 1 ? red[0] : 0.f);
+            r.cs[2 * t] = excl + a0;
+            r.cs[2 * t + 1] = excl + a1;
+            r.dt[2 * t] = dtv.x;
+            r.dt[2 * t + 1] = dtv.y;
+            if (t == 0) r.Dh = Dh;
+            named_bar_sync(kBarPrep, 64);
+            const float cs_end = r.cs[kT - 1];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int col = jb * 32 + q * 8;
-                uint8_t* dst = st + (col >> 6) * 16384 + sw128_offset(i, col & 63);
-                *reinterpret_cast<uint4*>(dst) =
-                    make_uint4(packed[q * 4], packed[q * 4 + 1], packed[q * 4 + 2], packed[q * 4 + 3]);
+            for (int e = 0; e < 2; ++e) {
+                const int j = 2 * t + e;
+                const float csj = r.cs[j];
+                const float dj = e ? dtv.y : dtv.x;
+                r.colf[j] = ex2_approx(r.cs[j | 31] - csj) * dj;
+                r.w[j] = ex2_approx(cs_end - csj) * dj;
             }
-        }
-    }
-    fence_async_shared();
-    tc_fence_before_sync();
-    __syncthreads();
+            named_bar_sync(kBarPrep, 64);
+            if (t == 0) mbar_arrive(bars + kFullRec + c);
 
-    // ---- MMA2: Yd = S~ X
-    if (tid == 0) {
-        tc_fence_after_sync();
-        const uint32_t st_base = smem_addr(sm + S::kSt);
-        const uint32_t x_base = smem_addr(sm + S::kX);
-        constexpr uint32_t id_y = idesc_bf16(128, kP, false, true);
+            // X~ = w o X (row j of the swizzled tile is the 128 bytes at j * 128)
+            wait_bar(bars + kFullX + xs, (k / kXStages) & 1, abort_flag, p.status);
+            wait_bar(bars + kEmptyXt, (k & 1) ^ 1, abort_flag, p.status);
+            {
+                const uint4* src = reinterpret_cast<const uint4*>(sm + Smem::kX + xs * kTileBytesX);
+                uint4* dst = reinterpret_cast<uint4*>(sm + Smem::kXt);
 #pragma unroll
-        for (int k = 0; k < kT / 16; ++k) {
-            mma_bf16(tmem + kColYd, sdesc_sw128(st_base + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
-                     sdesc_sw128(x_base + k * 2048, 16384, 1024), id_y, k > 0);
-        }
-        mma_commit(bar_mma2);
-    }
-
-    // ---- 4. look-back: the previous tile of this head publishes h_prev
-    const size_t PN = static_cast<size_t>(kP) * N;
-    if (tid == 0 && tile > 0) {
-        const unsigned int* f = p.flags + chain;
-        bool ok = false;
-        for (unsigned long long it = 0; it < p.wait_limit; ++it) {
-            if (ld_acquire_gpu(f) >= static_cast<unsigned int>(tile)) { ok = true; break; }
-            __nanosleep(64);
-        }
-        if (!ok) {
-            record_status(p.status, kDevWaitTimeout);
-            s_flag[0] = 1;
-        }
-    }
-    __syncthreads();
-
-    // thread n owns state rows n (and n + 128 for N = 256): 64 p values each
-    const float dec_tile = exp2f(cs_end);
-    const float* hsrc = nullptr;
-    if (tile == 0) {
-        hsrc = p.init ? p.init + static_cast<size_t>(chain) * PN : nullptr;
-    } else if (!s_flag[0]) {
-        hsrc = p.ring + (static_cast<size_t>(chain) * 2 + ((tile - 1) & 1)) * PN;
-    }
-    const bool last = tile == p.ntiles - 1;
-    float* hdst = last ? (p.final_state ? p.final_state + static_cast<size_t>(chain) * PN : nullptr)
-                       : p.ring + (static_cast<size_t>(chain) * 2 + (tile & 1)) * PN;
-#pragma unroll 1
-    for (int m = 0; m < N / 128; ++m) {
-        const int n = tid + m * 128;
-        float hp[kP];
+                for (int half = 0; half < 2; ++half) {
+                    uint4 v[8];
 #pragma unroll
-        for (int q = 0; q < kP; ++q)
-            hp[q] = hsrc ? __ldcg(hsrc + static_cast<size_t>(q) * N + n) : 0.f;
-        // h_prev (bf16) as the K-major B operand of MMA3: row p, column n
-        uint8_t* hs = sm + S::kHs + (n >> 6) * 8192;
+                    for (int q = 0; q < 8; ++q) v[q] = src[t + (half * 8 + q) * 64];
 #pragma unroll
-        for (int q = 0; q < kP; ++q)
-            *reinterpret_cast<__nv_bfloat16*>(hs + sw128_offset(q, n & 63)) = __float2bfloat16_rn(hp[q]);
-        // h = exp(cs_end) h_prev + s
-        float sv[32];
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            tmem_ld32(tmem + lane_off + kColState + m * 64 + half * 32, sv);
-            tmem_wait_ld();
-#pragma unroll
-            for (int q = 0; q < 32; ++q) {
-                const int pq = half * 32 + q;
-                const float hn = dec_tile * hp[pq] + sv[q];
-                if (hdst) hdst[static_cast<size_t>(pq) * N + n] = hn;
-            }
-        }
-    }
-    __threadfence();
-    fence_async_shared();
-    tc_fence_before_sync();
-    __syncthreads();
-    if (tid == 0 && !last && !p.skip_publish) st_release_gpu(p.flags + chain, tile + 1);
-
-    // ---- MMA3: Ys = C h_prev^T
-    if (tid == 0) {
-        tc_fence_after_sync();
-        const uint32_t c_base = smem_addr(sm + S::kC);
-        const uint32_t hs_base = smem_addr(sm + S::kHs);
-        constexpr uint32_t id_y = idesc_bf16(128, kP, false, false);
-#pragma unroll
-        for (int k = 0; k < N / 16; ++k) {
-            mma_bf16(tmem + kColYs, sdesc_sw128(c_base + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
-                     sdesc_sw128(hs_base + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024), id_y, k > 0);
-        }
-        mma_commit(bar_mma3);
-    }
-    bool ok2 = mbar_wait(bar_mma2, 0, kMbarLimit);
-    bool ok3 = mbar_wait(bar_mma3, 0, kMbarLimit);
-    if (!ok2 || !ok3) record_status(p.status, kDevWaitTimeout);
-    tc_fence_after_sync();
-
-    // ---- 5. epilogue: y_i = Yd_i + exp(cs_i) Ys_i + D x_i
-    {
-        const int i = tid;
-        const float Dh = p.D ? p.D[h] : 0.f;
-        const float ei = exp2f(cs_i);
-        const uint8_t* xrow = sm + S::kX;
-        __nv_bfloat16* yrow = p.y + ((static_cast<size_t>(b) * p.L + t0 + i) * p.H + h) * kP;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            float yd[32], ys[32];
-            tmem_ld32(tmem + lane_off + kColYd + half * 32, yd);
-            tmem_ld32(tmem + lane_off + kColYs + half * 32, ys);
-            tmem_wait_ld();
-            uint32_t out[16];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int col = half * 32 + q * 8;
-                const uint4 xq = *reinterpret_cast<const uint4*>(xrow + sw128_offset(i, col));
-                const uint32_t* xu = reinterpret_cast<const uint32_t*>(&xq);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 xf = unpack_bf16x2(xu[e]);
-                    const int c = q * 8 + e * 2;
-                    out[q * 4 + e] = pack_bf16x2(yd[c] + ei * ys[c] + Dh * xf.x,
-                                                 yd[c + 1] + ei * ys[c + 1] + Dh * xf.y);
+                    for (int q = 0; q < 8; ++q) {
+                        const int chunk = t + (half * 8 + q) * 64;
+                        dst[chunk] = scale_bf16x8(v[q], r.w[chunk >> 3]);
+                    }
                 }
             }
-            if (i < rows) {
-                uint4* dst = reinterpret_cast<uint4*>(yrow + half * 32);
+            fence_async_shared();
+            named_bar_sync(kBarPrep, 64);
+            if (t == 0) mbar_arrive(bars + kFullXt);
+        }
+    } else if (warp >= kWgMask0 && warp < kWgMask0 + 4) {
+        // ------------------------------------------- mask S -> S~ (in place, TMEM)
+        // S~ (bf16 pairs) overwrites the first 64 columns of the tile's S: block
+        // jb of S~ lands on columns 16 jb .. 16 jb + 15, which hold S values that
+        // were read before (blocks <= jb), so reads always stay ahead of writes.
+        const int wq = warp - kWgMask0;  // lane quadrant: rows 32 wq .. 32 wq + 31
+        const int i = wq * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+        Seq s;
+        s.begin(p);
+        for (int k = 0; s.valid; ++k, s.next(p)) {
+            const int c = k % kCsStages, sb = k & 1;
+            const TileRec& r = recs[c];
+            wait_bar(bars + kFullRec + c, (k / kCsStages) & 1, abort_flag, p.status);
+            wait_bar(bars + kFullS + sb, (k >> 1) & 1, abort_flag, p.status);
+            tc_fence_after_sync();
+            const float cs_i = r.cs[i];
+            const float Dh = r.Dh;
+            const uint32_t s_col = tmem + lane_off + kColS + sb * 128;
+#pragma unroll 1
+            for (int jb = 0; jb < 4; ++jb) {
+                uint32_t packed[16];
+                if (jb < wq) {
+                    // block wholly left of the diagonal: row factor x column factor
+                    float sv[32];
+                    tmem_ld32(s_col + jb * 32, sv);
+                    tmem_wait_ld();
+                    const float rf = ex2_approx(cs_i - r.cs[jb * 32 + 31]);
+                    const float4* cf = reinterpret_cast<const float4*>(r.colf + jb * 32);
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    dst[q] = make_uint4(out[q * 4], out[q * 4 + 1], out[q * 4 + 2], out[q * 4 + 3]);
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 f = cf[q];
+                        packed[q * 2] = pack_bf16x2(sv[q * 4] * f.x * rf, sv[q * 4 + 1] * f.y * rf);
+                        packed[q * 2 + 1] =
+                            pack_bf16x2(sv[q * 4 + 2] * f.z * rf, sv[q * 4 + 3] * f.w * rf);
+                    }
+                } else if (jb == wq) {
+                    // block on the diagonal. Every lane evaluates every term and the
+                    // position only selects values: rows diverge on j < i, and a
+                    // per-element branch would serialise the warp.
+                    float sv[32];
+                    tmem_ld32(s_col + jb * 32, sv);
+                    tmem_wait_ld();
+                    const float4* cs4 = reinterpret_cast<const float4*>(r.cs + jb * 32);
+                    const float4* dt4 = reinterpret_cast<const float4*>(r.dt + jb * 32);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 c4 = cs4[q];
+                        const float4 d4 = dt4[q];
+                        const float csj[4] = {c4.x, c4.y, c4.z, c4.w};
+                        const float dtj[4] = {d4.x, d4.y, d4.z, d4.w};
+                        float m[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int jj = q * 4 + e;
+                            const float below = sv[jj] * ex2_approx(fminf(cs_i - csj[e], 0.f)) * dtj[e];
+                            const float diag = fmaf(sv[jj], dtj[e], Dh);
+                            const float v = jj < lane ? below : 0.f;
+                            m[e] = jj == lane ? diag : v;
+                        }
+                        packed[q * 2] = pack_bf16x2(m[0], m[1]);
+                        packed[q * 2 + 1] = pack_bf16x2(m[2], m[3]);
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) packed[q] = 0u;
+                }
+                tmem_st16(s_col + jb * 16, packed);
+            }
+            tmem_wait_st();
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bars + kFullSt + sb);
+                mbar_arrive(bars + kEmptyRec + c);
+            }
+        }
+    } else if (warp >= kWgOut0 && warp < kWgOut0 + 4) {
+        // ------------------ h_prev operand, state, epilogue, look-back, publish
+        const int wq = warp - kWgOut0;
+        const int n = wq * 32 + lane;  // state row / tile row / TMEM lane
+        const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+        const size_t PN = static_cast<size_t>(kP) * kN;
+        float h[kP];
+        Seq s;
+        s.begin(p);
+        for (int k = 0; s.valid; ++k, s.next(p)) {
+            const bool first = s.tile == s.seg * p.seg_len;
+            const bool last = s.tile == s.tile_end - 1;
+            const int c = k % kCsStages, sb = k & 1;
+            if (first) {
+                // look-back: the state before this segment
+                if (s.seg == 0) {
+                    const float* src = p.init ? p.init + static_cast<size_t>(s.chain) * PN : nullptr;
+#pragma unroll
+                    for (int q = 0; q < kP; ++q) h[q] = src ? src[static_cast<size_t>(q) * kN + n] : 0.f;
+                } else {
+                    if (n == 0 && !*abort_flag) {
+                        const unsigned int* f = p.flags + s.chain;
+                        bool ok = false;
+                        const uint64_t t0 = global_timer_ns();
+                        for (unsigned long long it = 0; it < p.wait_limit; ++it) {
+                            if (ld_acquire_gpu(f) >= static_cast<unsigned int>(s.seg)) {
+                                ok = true;
+                                break;
+                            }
+                            if ((it & 255) == 255 && global_timer_ns() - t0 > 4000000000ull) break;
+                            __nanosleep(64);
+                        }
+                        if (!ok) {
+                            record_status(p.status, kDevWaitTimeout);
+                            *abort_flag = 1;
+                        }
+                    }
+                    named_bar_sync(kBarOut, 128);
+                    const float4* src = reinterpret_cast<const float4*>(
+                        p.ring + ((static_cast<size_t>(s.chain) * 2 + ((s.seg - 1) & 1)) * kN + n) * kP);
+#pragma unroll
+                    for (int q = 0; q < kP / 4; ++q) {
+                        const float4 v = __ldcg(src + q);
+                        h[q * 4 + 0] = v.x;
+                        h[q * 4 + 1] = v.y;
+                        h[q * 4 + 2] = v.z;
+                        h[q * 4 + 3] = v.w;
+                    }
+                }
+            }
+            const TileRec& r = recs[c];
+            wait_bar(bars + kFullRec + c, (k / kCsStages) & 1, abort_flag, p.status);
+            const float cs_n = r.cs[n];
+            const float dec = ex2_approx(r.cs[kT - 1]);
+
+            // the bf16 h_prev operand of MMA3 (row n of [N][P], MN-major)
+            wait_bar(bars + kEmptyHs, (k & 1) ^ 1, abort_flag, p.status);
+            {
+                uint8_t* row = sm + Smem::kHs + n * 128;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const uint4 v = make_uint4(pack_bf16x2(h[q * 8 + 0], h[q * 8 + 1]),
+                                               pack_bf16x2(h[q * 8 + 2], h[q * 8 + 3]),
+                                               pack_bf16x2(h[q * 8 + 4], h[q * 8 + 5]),
+                                               pack_bf16x2(h[q * 8 + 6], h[q * 8 + 7]));
+                    *reinterpret_cast<uint4*>(row + (((q ^ n) & 7) << 4)) = v;
+                }
+            }
+            fence_async_shared();
+            named_bar_sync(kBarOut, 128);
+            if (n == 0) mbar_arrive(bars + kFullHs);
+
+            // h = exp(cs_end) h_prev + s
+            wait_bar(bars + kFullStates + sb, (k >> 1) & 1, abort_flag, p.status);
+            tc_fence_after_sync();
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float sv[32];
+                tmem_ld32(tmem + lane_off + kColSt + sb * 64 + half * 32, sv);
+                tmem_wait_ld();
+#pragma unroll
+                for (int q = 0; q < 32; ++q) h[half * 32 + q] = dec * h[half * 32 + q] + sv[q];
+            }
+            tc_fence_before_sync();
+            named_bar_sync(kBarOut, 128);
+            if (n == 0) mbar_arrive(bars + kEmptyStates + sb);
+
+            if (last) {
+                if (s.tile == p.ntiles - 1) {
+                    if (p.final_state) {
+                        float* dst = p.final_state + static_cast<size_t>(s.chain) * PN;
+#pragma unroll
+                        for (int q = 0; q < kP; ++q) dst[static_cast<size_t>(q) * kN + n] = h[q];
+                    }
+                } else {
+                    float4* dst = reinterpret_cast<float4*>(
+                        p.ring + ((static_cast<size_t>(s.chain) * 2 + (s.seg & 1)) * kN + n) * kP);
+#pragma unroll
+                    for (int q = 0; q < kP / 4; ++q)
+                        dst[q] = make_float4(h[q * 4], h[q * 4 + 1], h[q * 4 + 2], h[q * 4 + 3]);
+                    __threadfence();
+                    named_bar_sync(kBarOut, 128);
+                    if (n == 0 && !p.skip_publish)
+                        st_release_gpu(p.flags + s.chain, static_cast<unsigned int>(s.seg + 1));
+                }
+            }
+
+            // epilogue: y_n = Yd_n + exp(cs_n) Ys_n (bf16)
+            wait_bar(bars + kFullY + sb, (k >> 1) & 1, abort_flag, p.status);
+            tc_fence_after_sync();
+            {
+                const int rows = min(kT, p.L - s.tile * kT);
+                const float en = ex2_approx(cs_n);
+                __nv_bfloat16* yrow =
+                    p.y + ((static_cast<size_t>(s.b) * p.L + s.tile * kT + n) * p.H + s.h) * kP;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    float yd[32], ys[32];
+                    tmem_ld32(tmem + lane_off + kColY + sb * 64 + half * 32, yd);
+                    tmem_ld32(tmem + lane_off + kColS + sb * 128 + 64 + half * 32, ys);
+                    tmem_wait_ld();
+                    if (n < rows) {
+                        uint4* dst = reinterpret_cast<uint4*>(yrow + half * 32);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint32_t o[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int c2 = q * 8 + e * 2;
+                                o[e] = pack_bf16x2(fmaf(en, ys[c2], yd[c2]),
+                                                   fmaf(en, ys[c2 + 1], yd[c2 + 1]));
+                            }
+                            dst[q] = make_uint4(o[0], o[1], o[2], o[3]);
+                        }
+                    }
+                }
+            }
+            tc_fence_before_sync();
+            named_bar_sync(kBarOut, 128);
+            if (n == 0) {
+                mbar_arrive(bars + kEmptyY + sb);
+                mbar_arrive(bars + kEmptyRec + c);
             }
         }
     }
 
     // ---- teardown
+    __syncwarp();
     tc_fence_before_sync();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+    if (warp == kWarpAlloc) tmem_dealloc(tmem, kTmemCols);
     if (tid == 0) {
         __threadfence();
         const unsigned int done = atomicAdd(p.ctrl + 1, 1u);
-        if (done == static_cast<unsigned int>(p.total) - 1u) {
+        if (done == gridDim.x - 1u) {
             // every other CTA has finished: leave the control words zeroed
             for (int c = 0; c < p.chains; ++c) p.flags[c] = 0u;
-            p.ctrl[0] = 0u;
             p.ctrl[1] = 0u;
             __threadfence();
         }
@@ -475,12 +762,21 @@ WsLayout ws_layout(const FwdArgs& a)
 
 int g_skip_publish = 0;
 
-template <int N>
+// Segments per chain: enough items for about eight per CTA, at least one tile each.
+void choose_segments(int ntiles, int chains, int ctas, int* seg_len, int* nseg)
+{
+    long long want = (8ll * ctas + chains - 1) / chains;
+    if (want < 1) want = 1;
+    if (want > ntiles) want = ntiles;
+    *seg_len = static_cast<int>((ntiles + want - 1) / want);
+    *nseg = (ntiles + *seg_len - 1) / *seg_len;
+}
+
 cudaError_t launch(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)
 {
     CUtensorMap tmX, tmB, tmC;
-    if (!make_map(&tmX, a.x, kP, a.H, a.L, a.B) || !make_map(&tmB, a.Bm, N, a.G, a.L, a.B) ||
-        !make_map(&tmC, a.Cm, N, a.G, a.L, a.B))
+    if (!make_map(&tmX, a.x, kP, a.H, a.L, a.B) || !make_map(&tmB, a.Bm, kN, a.G, a.L, a.B) ||
+        !make_map(&tmC, a.Cm, kN, a.G, a.L, a.B))
         return cudaErrorInvalidValue;
     const WsLayout w = ws_layout(a);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -500,16 +796,18 @@ cudaError_t launch(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)
     p.L = a.L;
     p.H = a.H;
     p.G = a.G;
-    p.N = N;
     p.ntiles = (a.L + kT - 1) / kT;
     p.chains = a.B * a.H;
-    p.total = p.ntiles * p.chains;
+    const int ctas_max = ctx.num_sms > 0 ? ctx.num_sms : 1;
+    choose_segments(p.ntiles, p.chains, ctas_max, &p.seg_len, &p.nseg);
+    p.items = p.chains * p.nseg;
     p.skip_publish = g_skip_publish;
-    const uint32_t smem = Smem<N>::kBytes;
-    cudaError_t e = cudaFuncSetAttribute(tc_forward_kernel<N>,
+    const int grid = p.items < ctas_max ? p.items : ctas_max;
+    const uint32_t smem = Smem::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(tc_forward_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    tc_forward_kernel<N><<<p.total, kThreads, smem, ctx.stream>>>(tmX, tmB, tmC, p);
+    tc_forward_kernel<<<grid, kThreads, smem, ctx.stream>>>(tmX, tmB, tmC, p);
     return cudaGetLastError();
 }
 
@@ -517,7 +815,7 @@ cudaError_t launch(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)
 
 bool tc_supported(const FwdArgs& a)
 {
-    return a.bf16 && a.P == kP && a.N == 128 && (a.chunk == 128 || a.chunk == 256) &&
+    return a.bf16 && a.P == kP && a.N == kN && (a.chunk == 128 || a.chunk == 256) &&
            static_cast<long long>(a.B) * a.L > 0 &&
            static_cast<long long>((a.L + kT - 1) / kT) * a.B * a.H < (1ll << 31);
 }
@@ -530,10 +828,8 @@ void tc_set_skip_publish(int v) { g_skip_publish = v; }
 
 cudaError_t tc_forward(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)
 {
-    switch (a.N) {
-    case 128: return launch<128>(a, workspace, ctx);
-    default: return cudaErrorInvalidValue;
-    }
+    if (!tc_supported(a)) return cudaErrorInvalidValue;
+    return launch(a, workspace, ctx);
 }
 
 }  // namespace ssd
