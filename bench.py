@@ -56,6 +56,17 @@ def algorithmic_flops(w: gen.Workload) -> int:
     return BL * w.H * (w.chunk * w.P + 4 * w.N * w.P) + BL * w.G * w.chunk * w.N
 
 
+def combine_ranks(local_ms: float, tokens_per_rank: int, world: int, dist=None, device=None):
+    """Max of the per-rank step times (the slowest rank bounds the job) and the
+    whole-job throughput in Mtokens/s. Only timings cross ranks; no data does."""
+    import torch
+    t = torch.tensor([local_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    return ms, tokens_per_rank * world / (ms / 1e3) / 1e6
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -248,15 +259,13 @@ def run_ours(args):
         barrier()
     ssd.poll_status(stream)
     per_step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    ms_local = statistics.mean(per_step_ms)
-    t = torch.tensor([ms_local], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
+    ms, _ = combine_ranks(statistics.mean(per_step_ms), w.tokens, world, dist, dev)
+    decode = time_decode(ssd, dev, flush, args.warmup, args.steps, world, dist)
 
     # end to end through the host-buffer entry point: H2D inputs, forward, D2H y + state
     if args.no_e2e:
-        return _report(args, w, rank, world, ms, per_step_ms, clk, inp, None, host, ssd, code, dist)
+        return _report(args, w, rank, world, ms, per_step_ms, clk, inp, None, host, ssd, code, dist,
+                       decode)
     pin = {k: v.pin_memory() for k, v in host.items()}
     y_host = torch.empty_like(host["x"]).pin_memory()
     fs_host = torch.empty((w.B, w.H, w.P, w.N), dtype=torch.float32).pin_memory()
@@ -278,15 +287,46 @@ def run_ours(args):
         e2e_step()
     e_end.record(stream)
     barrier()
-    e2e_ms = e_start.elapsed_time(e_end) / e2e_steps
-    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_ms = float(t.item())
-    return _report(args, w, rank, world, ms, per_step_ms, clk, inp, e2e_ms, host, ssd, code, dist)
+    e2e_ms, _ = combine_ranks(e_start.elapsed_time(e_end) / e2e_steps, w.tokens, world, dist, dev)
+    return _report(args, w, rank, world, ms, per_step_ms, clk, inp, e2e_ms, host, ssd, code, dist,
+                   decode)
 
 
-def _report(args, w, rank, world, ms, per_step_ms, clk, inp, e2e_ms, host, ssd, code, dist):
+def time_decode(ssd, dev, flush, warmup, steps, world, dist):
+    """ssd_step on the decode workload (one token for each of B sequences from a
+    random fp32 state), L2 flushed between steps outside the events."""
+    import torch
+    d = gen.DECODE
+    s = gen.make_step_inputs(d["B"], d["H"], d["P"], d["G"], d["N"], d["dtype"], seed=5)
+    io = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
+    x, Bm, Cm = io(s.x), io(s.Bm), io(s.Cm)
+    dt, A, D = (torch.from_numpy(v).to(dev) for v in (s.dt, s.A, s.D))
+    state = torch.from_numpy(s.state).to(dev)
+    y = torch.empty_like(x)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        flush.zero_()
+        ssd.step(x, dt, A, Bm, Cm, D, state, y=y, stream=stream)
+    times = []
+    for _ in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        ssd.step(x, dt, A, Bm, Cm, D, state, y=y, stream=stream)
+        e1.record(stream)
+        times.append((e0, e1))
+    ssd.poll_status(stream)
+    ms, _ = combine_ranks(statistics.mean(a.elapsed_time(b) for a, b in times), d["B"], world,
+                          dist, dev)
+    nbytes = (2 * d["B"] * d["H"] * d["P"] * d["N"] * 4 + 2 * d["B"] * d["H"] * d["P"] * 2
+              + d["B"] * d["H"] * 4 + 2 * d["B"] * d["G"] * d["N"] * 2 + 2 * d["H"] * 4)
+    return {"workload": d["name"], "ms_per_step": ms,
+            "value": d["B"] * world / (ms / 1e3) / 1e6, "unit": "Mtokens/s",
+            "algorithmic_bytes": nbytes, "achieved_gbs": nbytes / (ms / 1e3) / 1e9}
+
+
+def _report(args, w, rank, world, ms, per_step_ms, clk, inp, e2e_ms, host, ssd, code, dist,
+            decode=None):
     tokens_all = w.tokens * world
     value = tokens_all / (ms / 1e3) / 1e6
     h2d = sum(v.numel() * v.element_size() for v in host.values())
@@ -338,6 +378,9 @@ def _report(args, w, rank, world, ms, per_step_ms, clk, inp, e2e_ms, host, ssd, 
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms, "api": "ssd_forward_host (pinned host buffers)"},
             "gpu_launches": launches * args.steps,
+            "decode": None if decode is None else dict(
+                decode, frac=decode["achieved_gbs"] / hbm_peak, bound="hbm",
+                peak=hbm_peak, peak_unit="GB/s"),
             "per_step_ms": {"min": min(per_step_ms), "median": statistics.median(per_step_ms),
                             "max": max(per_step_ms)},
         }

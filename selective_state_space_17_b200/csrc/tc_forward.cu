@@ -34,18 +34,17 @@
 // boundary does h travel through the workspace (a two-slot fp32 ring per
 // chain, published with a release flag and read after a bounded acquire poll).
 //
-// Warp roles inside the CTA (384 threads), linked by full/empty mbarrier rings
+// Warp roles inside the CTA (416 threads), linked by full/empty mbarrier rings
 // whose waits sleep rather than spin:
-//   warp 0        TMA producer: C, B (2 stages), X (3 stages), L2 prefetch of
-//                 the X tiles further ahead
-//   warp 1        MMA issuer, one tile of lag: MMA1 and states of tile k are
-//                 issued before MMA2 and MMA3 of tile k-1, so the tensor core
-//                 works on tile k while tile k-1 is being masked (S is double
-//                 buffered in TMEM)
-//   warps 2-3     tile prologue: cumsum, column factors, w o X
-//   warps 4-7     mask S -> S~
-//   warps 8-11    h_prev -> bf16 operand, state update, epilogue, look-back
-//                 and segment publication
+//   warp 0        TMA producer: C, B (2 stages), X (2 stages, one tile ahead),
+//                 L2 prefetch of the X tiles further ahead; TMEM allocation
+//   warp 1        MMA stream A: MMA1 and states of each tile
+//   warp 2        MMA stream B: MMA2 and MMA3 of each tile (S is double
+//                 buffered in TMEM, so stream A runs a tile ahead of stream B)
+//   warps 3, 12   tile prologue: cumsum, column factors, w o X
+//   warps 4-7     mask S -> S~, in place in TMEM
+//   warps 8-11    h_prev -> bf16 operand, state update, epilogue through a
+//                 TMA store, look-back and segment publication
 //
 // A chunk of 256 tokens is evaluated as two 128-token tiles: its quadratic
 // form split into 2 x 2 blocks, the diagonal blocks computed directly and the
@@ -72,18 +71,20 @@ constexpr int kN = 128;   // state dim on this path
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint64_t kMbarLimit = 1ull << 22;  // polls; each wait is also capped at ~2 s
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 416;
 constexpr int kWarpProducer = 0;
-constexpr int kWarpMma = 1;
-constexpr int kWarpPrep0 = 2;  // warps 2..3
-constexpr int kWarpAlloc = 2;
+constexpr int kWarpMmaA = 1;   // MMA1 and states
+constexpr int kWarpMmaB = 2;   // MMA2 and MMA3
+constexpr int kWarpPrepA = 3;  // prologue: warps 3 and 12
+constexpr int kWarpPrepB = 12;
+constexpr int kWarpAlloc = 0;
 constexpr int kWgMask0 = 4;    // warps 4..7
 constexpr int kWgOut0 = 8;     // warps 8..11
 constexpr int kBarPrep = 1;    // named barrier ids
 constexpr int kBarOut = 2;
 
 constexpr int kCbStages = 2;
-constexpr int kXStages = 3;
+constexpr int kXStages = 2;
 constexpr int kCsStages = 4;
 constexpr int kPrefetchAhead = 4;
 
@@ -134,7 +135,8 @@ struct Smem {
     static constexpr uint32_t kX = kB + kCbStages * kTileBytesCB;       // 3 x 16 KB
     static constexpr uint32_t kXt = kX + kXStages * kTileBytesX;        // 16 KB
     static constexpr uint32_t kHs = kXt + kTileBytesX;                  // N x 64 bf16
-    static constexpr uint32_t kRec = kHs + kN * kP * 2;                 // 4 x TileRec
+    static constexpr uint32_t kYs = kHs + kN * kP * 2;                  // y staging, 16 KB
+    static constexpr uint32_t kRec = kYs + kT * kP * 2;                 // 4 x TileRec
     static constexpr uint32_t kRed = kRec + kCsStages * sizeof(TileRec);  // 8 floats
     static constexpr uint32_t kBars = kRed + 32;
     static constexpr int kNumBars = 40;
@@ -148,7 +150,7 @@ static_assert(Smem::kBytes <= 227 * 1024, "shared memory budget");
 // mbarrier indices
 enum Bar : int {
     kFullCB = 0,      // 2
-    kEmptyCB = 2,     // 2: the commit after MMA3 frees C and B of the stage
+    kEmptyCB = 2,     // 2 (two arrivals: after states, after MMA3)
     kFullX = 4,       // 3
     kEmptyX = 7,      // 3
     kFullXt = 10,
@@ -202,22 +204,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__device__ __forceinline__ float2 unpack_bf16x2(uint32_t u)
-{
-    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
-}
-
-__device__ __forceinline__ uint4 scale_bf16x8(uint4 q, float f)
-{
-    uint32_t* u = reinterpret_cast<uint32_t*>(&q);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const float2 v = unpack_bf16x2(u[e]);
-        u[e] = pack_bf16x2(v.x * f, v.y * f);
-    }
-    return q;
-}
-
 // Bounded wait that turns a give-up into the CTA's abort mode: from then on
 // waits return at once, every role runs to the end of its loop on whatever is
 // in its buffers, and the device status word reports the timeout.
@@ -233,7 +219,8 @@ __device__ __forceinline__ void wait_bar(uint64_t* bar, uint32_t parity, volatil
 
 __global__ void __launch_bounds__(kThreads, 1)
 tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
-                  const __grid_constant__ CUtensorMap tmC, TcParams p)
+                  const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY,
+                  TcParams p)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte alignment for the swizzle atoms, by offsetting the shared array
@@ -252,9 +239,11 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         prefetch_tensormap(&tmX);
         prefetch_tensormap(&tmB);
         prefetch_tensormap(&tmC);
+        prefetch_tensormap(&tmY);
         for (int i = 0; i < Smem::kNumBars; ++i)
             mbar_init(bars + i, (i >= kEmptyRec && i < kEmptyRec + kCsStages) ? 5u
                                 : (i >= kFullSt && i < kFullSt + 2)          ? 4u
+                                : (i >= kEmptyCB && i < kEmptyCB + 2)        ? 2u
                                                                              : 1u);
         mbar_fence_init();
         *abort_flag = 0;
@@ -313,90 +302,85 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             for (int j = max(0, kx - kXStages); j < kx; ++j)
                 mbar_wait(bars + kFullX + j % kXStages, (j / kXStages) & 1, kMbarLimit);
         }
-    } else if (warp == kWarpMma) {
-        // ----------------------------------------------- all MMAs, one tile of lag
-        // per iteration: MMA1 of tile k, MMA2 + MMA3 of tile k-1, states of tile k
+    } else if (warp == kWarpMmaA) {
+        // ---------------------------------------------- stream A: MMA1, states
         if (lane == 0) {
             constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
             constexpr uint32_t id_st = idesc_bf16(128, kP, true, true);
-            constexpr uint32_t id_y2 = idesc_bf16(128, kP, false, true);
             const uint32_t xt_base = smem_addr(sm + Smem::kXt);
-            const uint32_t hs_base = smem_addr(sm + Smem::kHs);
             Seq s;
             s.begin(p);
-            int k = 0;
-            bool prev = false;
-            for (;;) {
-                const bool cur = s.valid;
-                if (cur) {
-                    const int cb = k % kCbStages, sb = k & 1;
-                    const uint32_t c_base = smem_addr(sm + Smem::kC + cb * kTileBytesCB);
-                    const uint32_t b_base = smem_addr(sm + Smem::kB + cb * kTileBytesCB);
-                    wait_bar(bars + kFullCB + cb, (k / kCbStages) & 1, abort_flag, p.status);
-                    // S[sb] held S~ and Ys of tile k-2 until its epilogue read them
-                    if (k >= 2) wait_bar(bars + kEmptyY + sb, ((k - 2) >> 1) & 1, abort_flag, p.status);
-                    tc_fence_after_sync();
+            for (int k = 0; s.valid; ++k, s.next(p)) {
+                const int cb = k % kCbStages, sb = k & 1;
+                const uint32_t c_base = smem_addr(sm + Smem::kC + cb * kTileBytesCB);
+                const uint32_t b_base = smem_addr(sm + Smem::kB + cb * kTileBytesCB);
+                wait_bar(bars + kFullCB + cb, (k / kCbStages) & 1, abort_flag, p.status);
+                // S[sb] held S~ and Ys of tile k-2 until its epilogue read them
+                if (k >= 2) wait_bar(bars + kEmptyY + sb, ((k - 2) >> 1) & 1, abort_flag, p.status);
+                tc_fence_after_sync();
 #pragma unroll
-                    for (int q = 0; q < kN / 16; ++q) {
-                        const uint32_t off = (q >> 2) * 16384 + (q & 3) * 32;
-                        mma_bf16(tmem + kColS + sb * 128, sdesc_sw128(c_base + off, 16, 1024),
-                                 sdesc_sw128(b_base + off, 16, 1024), id_s, q > 0);
-                    }
-                    mma_commit(bars + kFullS + sb);
+                for (int q = 0; q < kN / 16; ++q) {
+                    const uint32_t off = (q >> 2) * 16384 + (q & 3) * 32;
+                    mma_bf16(tmem + kColS + sb * 128, sdesc_sw128(c_base + off, 16, 1024),
+                             sdesc_sw128(b_base + off, 16, 1024), id_s, q > 0);
                 }
-                if (prev) {
-                    const int j = k - 1;
-                    const int cb = j % kCbStages, xs = j % kXStages, sb = j & 1;
-                    const uint32_t c_base = smem_addr(sm + Smem::kC + cb * kTileBytesCB);
-                    const uint32_t x_base = smem_addr(sm + Smem::kX + xs * kTileBytesX);
-                    wait_bar(bars + kFullSt + sb, (j >> 1) & 1, abort_flag, p.status);
-                    wait_bar(bars + kEmptyY + sb, ((j >> 1) & 1) ^ 1, abort_flag, p.status);
-                    tc_fence_after_sync();
+                mma_commit(bars + kFullS + sb);
+                wait_bar(bars + kEmptyStates + sb, ((k >> 1) & 1) ^ 1, abort_flag, p.status);
+                wait_bar(bars + kFullXt, k & 1, abort_flag, p.status);
+                tc_fence_after_sync();
 #pragma unroll
-                    for (int q = 0; q < kT / 16; ++q) {
-                        mma_bf16_tmem_a(tmem + kColY + sb * 64, tmem + kColS + sb * 128 + q * 8,
-                                        sdesc_sw128(x_base + q * 2048, 16384, 1024), id_y2, q > 0);
-                    }
-                    wait_bar(bars + kFullHs, j & 1, abort_flag, p.status);
-                    tc_fence_after_sync();
-#pragma unroll
-                    for (int q = 0; q < kN / 16; ++q) {
-                        mma_bf16(tmem + kColS + sb * 128 + 64,
-                                 sdesc_sw128(c_base + (q >> 2) * 16384 + (q & 3) * 32, 16, 1024),
-                                 sdesc_sw128(hs_base + q * 2048, 16384, 1024), id_y2, q > 0);
-                    }
-                    mma_commit(bars + kFullY + sb);
-                    mma_commit(bars + kEmptyHs);
-                    mma_commit(bars + kEmptyX + xs);
-                    mma_commit(bars + kEmptyCB + cb);
+                for (int q = 0; q < kT / 16; ++q) {
+                    mma_bf16(tmem + kColSt + sb * 64, sdesc_sw128(b_base + q * 2048, 16384, 1024),
+                             sdesc_sw128(xt_base + q * 2048, 16384, 1024), id_st, q > 0);
                 }
-                if (cur) {
-                    const int cb = k % kCbStages, sb = k & 1;
-                    const uint32_t b_base = smem_addr(sm + Smem::kB + cb * kTileBytesCB);
-                    wait_bar(bars + kEmptyStates + sb, ((k >> 1) & 1) ^ 1, abort_flag, p.status);
-                    wait_bar(bars + kFullXt, k & 1, abort_flag, p.status);
-                    tc_fence_after_sync();
-#pragma unroll
-                    for (int q = 0; q < kT / 16; ++q) {
-                        mma_bf16(tmem + kColSt + sb * 64,
-                                 sdesc_sw128(b_base + q * 2048, 16384, 1024),
-                                 sdesc_sw128(xt_base + q * 2048, 16384, 1024), id_st, q > 0);
-                    }
-                    mma_commit(bars + kEmptyXt);
-                    mma_commit(bars + kFullStates + sb);
-                }
-                if (!cur) break;
-                prev = true;
-                ++k;
-                s.next(p);
+                mma_commit(bars + kEmptyXt);
+                mma_commit(bars + kFullStates + sb);
+                mma_commit(bars + kEmptyCB + cb);
             }
             mma_commit(bars + kDrain);
             mbar_wait(bars + kDrain, 0, kMbarLimit);
         }
-    } else if (warp >= kWarpPrep0 && warp < kWarpPrep0 + 2) {
+    } else if (warp == kWarpMmaB) {
+        // ----------------------------------------------- stream B: MMA2, MMA3
+        if (lane == 0) {
+            constexpr uint32_t id_y2 = idesc_bf16(128, kP, false, true);
+            const uint32_t hs_base = smem_addr(sm + Smem::kHs);
+            Seq s;
+            s.begin(p);
+            for (int k = 0; s.valid; ++k, s.next(p)) {
+                const int cb = k % kCbStages, xs = k % kXStages, sb = k & 1;
+                const uint32_t c_base = smem_addr(sm + Smem::kC + cb * kTileBytesCB);
+                const uint32_t x_base = smem_addr(sm + Smem::kX + xs * kTileBytesX);
+                wait_bar(bars + kFullSt + sb, (k >> 1) & 1, abort_flag, p.status);
+                wait_bar(bars + kEmptyY + sb, ((k >> 1) & 1) ^ 1, abort_flag, p.status);
+                wait_bar(bars + kFullX + xs, (k / kXStages) & 1, abort_flag, p.status);
+                tc_fence_after_sync();
+#pragma unroll
+                for (int q = 0; q < kT / 16; ++q) {
+                    mma_bf16_tmem_a(tmem + kColY + sb * 64, tmem + kColS + sb * 128 + q * 8,
+                                    sdesc_sw128(x_base + q * 2048, 16384, 1024), id_y2, q > 0);
+                }
+                wait_bar(bars + kFullCB + cb, (k / kCbStages) & 1, abort_flag, p.status);
+                wait_bar(bars + kFullHs, k & 1, abort_flag, p.status);
+                tc_fence_after_sync();
+#pragma unroll
+                for (int q = 0; q < kN / 16; ++q) {
+                    mma_bf16(tmem + kColS + sb * 128 + 64,
+                             sdesc_sw128(c_base + (q >> 2) * 16384 + (q & 3) * 32, 16, 1024),
+                             sdesc_sw128(hs_base + q * 2048, 16384, 1024), id_y2, q > 0);
+                }
+                mma_commit(bars + kFullY + sb);
+                mma_commit(bars + kEmptyHs);
+                mma_commit(bars + kEmptyX + xs);
+                mma_commit(bars + kEmptyCB + cb);
+            }
+            mma_commit(bars + kDrain + 1);
+            mbar_wait(bars + kDrain + 1, 0, kMbarLimit);
+        }
+    } else if (warp == kWarpPrepA || warp == kWarpPrepB) {
         // ------------------------------------- prologue: cumsum, factors, w o X
-        const int t = tid - kWarpPrep0 * 32;  // 0..63, tokens 2t and 2t + 1
-        const int wq = warp - kWarpPrep0;
+        const int wq = warp == kWarpPrepA ? 0 : 1;
+        const int t = wq * 32 + lane;  // 0..63, tokens 2t and 2t + 1
         float* red = reinterpret_cast<float*>(sm + Smem::kRed);
         Seq s;
         s.begin(p);
@@ -464,7 +448,11 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         const int chunk = t + (half * 8 + q) * 64;
-                        dst[chunk] = scale_bf16x8(v[q], r.w[chunk >> 3]);
+                        const __nv_bfloat162 w2 = __float2bfloat162_rn(r.w[chunk >> 3]);
+                        __nv_bfloat162* e = reinterpret_cast<__nv_bfloat162*>(&v[q]);
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) e[u] = __hmul2(e[u], w2);
+                        dst[chunk] = v[q];
                     }
                 }
             }
@@ -556,6 +544,23 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
         const size_t PN = static_cast<size_t>(kP) * kN;
         float h[kP];
+        // the bf16 h_prev operand of MMA3 for tile kk (row n of [N][P],
+        // MN-major), once MMA3 of tile kk - 1 has read the previous one
+        auto write_hs = [&](int kk) {
+            wait_bar(bars + kEmptyHs, (kk & 1) ^ 1, abort_flag, p.status);
+            uint8_t* row = sm + Smem::kHs + n * 128;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const uint4 v = make_uint4(pack_bf16x2(h[q * 8 + 0], h[q * 8 + 1]),
+                                           pack_bf16x2(h[q * 8 + 2], h[q * 8 + 3]),
+                                           pack_bf16x2(h[q * 8 + 4], h[q * 8 + 5]),
+                                           pack_bf16x2(h[q * 8 + 6], h[q * 8 + 7]));
+                *reinterpret_cast<uint4*>(row + (((q ^ n) & 7) << 4)) = v;
+            }
+            fence_async_shared();
+            named_bar_sync(kBarOut, 128);
+            if (n == 0) mbar_arrive(bars + kFullHs);
+        };
         Seq s;
         s.begin(p);
         for (int k = 0; s.valid; ++k, s.next(p)) {
@@ -603,23 +608,7 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             wait_bar(bars + kFullRec + c, (k / kCsStages) & 1, abort_flag, p.status);
             const float cs_n = r.cs[n];
             const float dec = ex2_approx(r.cs[kT - 1]);
-
-            // the bf16 h_prev operand of MMA3 (row n of [N][P], MN-major)
-            wait_bar(bars + kEmptyHs, (k & 1) ^ 1, abort_flag, p.status);
-            {
-                uint8_t* row = sm + Smem::kHs + n * 128;
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const uint4 v = make_uint4(pack_bf16x2(h[q * 8 + 0], h[q * 8 + 1]),
-                                               pack_bf16x2(h[q * 8 + 2], h[q * 8 + 3]),
-                                               pack_bf16x2(h[q * 8 + 4], h[q * 8 + 5]),
-                                               pack_bf16x2(h[q * 8 + 6], h[q * 8 + 7]));
-                    *reinterpret_cast<uint4*>(row + (((q ^ n) & 7) << 4)) = v;
-                }
-            }
-            fence_async_shared();
-            named_bar_sync(kBarOut, 128);
-            if (n == 0) mbar_arrive(bars + kFullHs);
+            write_hs(k);
 
             // h = exp(cs_end) h_prev + s
             wait_bar(bars + kFullStates + sb, (k >> 1) & 1, abort_flag, p.status);
@@ -656,44 +645,49 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 }
             }
 
-            // epilogue: y_n = Yd_n + exp(cs_n) Ys_n (bf16)
+            // epilogue: y_n = Yd_n + exp(cs_n) Ys_n (bf16), staged in shared memory
+            // (128-byte swizzle) and written by one TMA store, which also clips
+            // the rows of a ragged last tile
             wait_bar(bars + kFullY + sb, (k >> 1) & 1, abort_flag, p.status);
+            if (n == 0) tma_store_wait_read();  // previous tile's store has read the stage
+            named_bar_sync(kBarOut, 128);
             tc_fence_after_sync();
             {
-                const int rows = min(kT, p.L - s.tile * kT);
                 const float en = ex2_approx(cs_n);
-                __nv_bfloat16* yrow =
-                    p.y + ((static_cast<size_t>(s.b) * p.L + s.tile * kT + n) * p.H + s.h) * kP;
+                uint8_t* yrow = sm + Smem::kYs + n * 128;
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float yd[32], ys[32];
-                    tmem_ld32(tmem + lane_off + kColY + sb * 64 + half * 32, yd);
-                    tmem_ld32(tmem + lane_off + kColS + sb * 128 + 64 + half * 32, ys);
+                for (int qd = 0; qd < 4; ++qd) {
+                    float yd[16], ys[16];
+                    tmem_ld16(tmem + lane_off + kColY + sb * 64 + qd * 16, yd);
+                    tmem_ld16(tmem + lane_off + kColS + sb * 128 + 64 + qd * 16, ys);
                     tmem_wait_ld();
-                    if (n < rows) {
-                        uint4* dst = reinterpret_cast<uint4*>(yrow + half * 32);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint32_t o[4];
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        uint32_t o[4];
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int c2 = q * 8 + e * 2;
-                                o[e] = pack_bf16x2(fmaf(en, ys[c2], yd[c2]),
-                                                   fmaf(en, ys[c2 + 1], yd[c2 + 1]));
-                            }
-                            dst[q] = make_uint4(o[0], o[1], o[2], o[3]);
+                        for (int e = 0; e < 4; ++e) {
+                            const int c2 = h2 * 8 + e * 2;
+                            o[e] = pack_bf16x2(fmaf(en, ys[c2], yd[c2]), fmaf(en, ys[c2 + 1], yd[c2 + 1]));
                         }
+                        const int chunk = qd * 2 + h2;
+                        *reinterpret_cast<uint4*>(yrow + (((chunk ^ n) & 7) << 4)) =
+                            make_uint4(o[0], o[1], o[2], o[3]);
                     }
                 }
             }
+            fence_async_shared();
             tc_fence_before_sync();
             named_bar_sync(kBarOut, 128);
             if (n == 0) {
+                tma_store_4d(&tmY, sm + Smem::kYs, 0, s.h, s.tile * kT, s.b);
+                tma_store_commit();
                 mbar_arrive(bars + kEmptyY + sb);
                 mbar_arrive(bars + kEmptyRec + c);
             }
         }
     }
+
+    if (warp == kWgOut0 && lane == 0) tma_store_wait_all();
 
     // ---- teardown
     __syncwarp();
@@ -774,9 +768,9 @@ void choose_segments(int ntiles, int chains, int ctas, int* seg_len, int* nseg)
 
 cudaError_t launch(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)
 {
-    CUtensorMap tmX, tmB, tmC;
+    CUtensorMap tmX, tmB, tmC, tmY;
     if (!make_map(&tmX, a.x, kP, a.H, a.L, a.B) || !make_map(&tmB, a.Bm, kN, a.G, a.L, a.B) ||
-        !make_map(&tmC, a.Cm, kN, a.G, a.L, a.B))
+        !make_map(&tmC, a.Cm, kN, a.G, a.L, a.B) || !make_map(&tmY, a.y, kP, a.H, a.L, a.B))
         return cudaErrorInvalidValue;
     const WsLayout w = ws_layout(a);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -807,7 +801,7 @@ cudaError_t launch(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)
     cudaError_t e = cudaFuncSetAttribute(tc_forward_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    tc_forward_kernel<<<grid, kThreads, smem, ctx.stream>>>(tmX, tmB, tmC, p);
+    tc_forward_kernel<<<grid, kThreads, smem, ctx.stream>>>(tmX, tmB, tmC, tmY, p);
     return cudaGetLastError();
 }
 
