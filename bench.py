@@ -67,6 +67,23 @@ def combine_ranks(local_ms: float, tokens_per_rank: int, world: int, dist=None, 
     return ms, tokens_per_rank * world / (ms / 1e3) / 1e6
 
 
+def recorded_traffic(workload: str):
+    """DRAM bytes (read + write) of one launch from the ncu capture recorded in
+    profiles/traffic.json, or None when the kernel source has changed since."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f).get(workload)
+        if not rec:
+            return None
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
+                return None
+        return rec["traffic_bytes"]
+    except (OSError, ValueError, KeyError):
+        return None
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -342,14 +359,7 @@ def _report(args, w, rank, world, ms, per_step_ms, clk, inp, e2e_ms, host, ssd, 
     t_tc = flops / (tc_peak * 1e12)
     bound = "hbm" if t_hbm >= t_tc else "tensor"
     launches = ssd.kernel_count(w.B, w.L, w.H, w.P, w.G, w.N, w.chunk, code)
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tpath):
-        try:
-            with open(tpath) as f:
-                traffic = json.load(f).get(w.name)
-        except (OSError, ValueError):
-            traffic = None
+    traffic = recorded_traffic(w.name)
 
     result = None
     if rank == 0:
