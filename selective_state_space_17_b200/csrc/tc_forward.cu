@@ -36,11 +36,15 @@
 //
 // Warp roles inside the CTA (416 threads), linked by full/empty mbarrier rings
 // whose waits sleep rather than spin:
-//   warp 0        TMA producer: C, B (2 stages), X (2 stages, one tile ahead),
-//                 L2 prefetch of the X tiles further ahead; TMEM allocation
+//   warp 0        TMA producer: C, B (2 stages) and X (2 stages) as two
+//                 independent streams, L2 prefetch of the X tiles further
+//                 ahead; TMEM allocation
 //   warp 1        MMA stream A: MMA1 and states of each tile
 //   warp 2        MMA stream B: MMA2 and MMA3 of each tile (S is double
 //                 buffered in TMEM, so stream A runs a tile ahead of stream B)
+// The producer and MMA warps run their loops warp-wide and issue from one
+// elected lane, with the shared-memory descriptors built once per stage (a K
+// step only moves the start address), which keeps the issue path short.
 //   warps 3, 12   tile prologue: cumsum, column factors, w o X
 //   warps 4-7     mask S -> S~, in place in TMEM
 //   warps 8-11    h_prev -> bf16 operand, state update, epilogue through a
@@ -173,7 +177,7 @@ struct Seq {
     int item, tile, tile_end, seg, chain, b, h;
     bool valid;
 
-    __device__ void setup(const TcParams& p)
+    __device__ __noinline__ void setup(const TcParams& p)
     {
         valid = item < p.items;
         if (!valid) return;
@@ -207,14 +211,25 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 // Bounded wait that turns a give-up into the CTA's abort mode: from then on
 // waits return at once, every role runs to the end of its loop on whatever is
 // in its buffers, and the device status word reports the timeout.
+__device__ __noinline__ void wait_gave_up(volatile int* abort_flag, unsigned int* status)
+{
+    record_status(status, kDevWaitTimeout);
+    *abort_flag = 1;
+}
+
+// Bounded wait (polls, each of which may sleep; the clock is read every 256
+// polls). The give-up path is out of line: it runs at most once per CTA.
 __device__ __forceinline__ void wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                         unsigned int* status)
 {
     if (*abort_flag) return;
-    if (!mbar_wait(bar, parity, kMbarLimit)) {
-        record_status(status, kDevWaitTimeout);
-        *abort_flag = 1;
+    if (mbar_try_wait(bar, parity)) return;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return;
+        if ((it & 255u) == 0u && (it >= kMbarLimit || global_timer_ns() - t0 > 2000000000ull)) break;
     }
+    wait_gave_up(abort_flag, status);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -259,124 +274,168 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
 
     if (warp == kWarpProducer) {
         // ------------------------------------------------------------- producer
-        if (lane == 0) {
-            Seq s, pf;
-            s.begin(p);
-            pf.begin(p);
-            for (int d = 0; d < kPrefetchAhead && pf.valid; ++d) pf.next(p);
-            // X runs one tile ahead of C and B: its stage frees earlier
-            Seq sx = s;
-            auto load_x = [&](int kx) {
-                const int xs = kx % kXStages;
-                wait_bar(bars + kEmptyX + xs, ((kx / kXStages) & 1) ^ 1, abort_flag, p.status);
-                mbar_arrive_expect_tx(bars + kFullX + xs, kTileBytesX);
-                tma_load_4d(sm + Smem::kX + xs * kTileBytesX, &tmX, 0, sx.h, sx.tile * kT, sx.b,
-                            bars + kFullX + xs);
-                sx.next(p);
-            };
-            int kx = 0;
-            if (sx.valid) load_x(kx++);
-            int k = 0;
-            for (; s.valid; ++k, s.next(p)) {
-                if (pf.valid) {
-                    tma_prefetch_l2_4d(&tmX, 0, pf.h, pf.tile * kT, pf.b);
-                    pf.next(p);
-                }
-                const int g = s.h / (p.H / p.G);
-                const int t0 = s.tile * kT;
+        // Two independent load streams, C/B (2 stages) and X (2 stages), each in
+        // tile order: the warp polls both stage rings and issues whichever is
+        // free, so a late X stage never holds back the next C/B tile. One
+        // elected lane issues; the whole warp polls.
+        Seq s, sx, pf;
+        s.begin(p);
+        sx = s;
+        pf = s;
+        for (int d = 0; d < kPrefetchAhead && pf.valid; ++d) pf.next(p);
+        int k = 0, kx = 0;
+        uint64_t idle_since = 0;
+        while (s.valid || sx.valid) {
+            if (*abort_flag) break;
+            bool issued = false;
+            if (s.valid) {
                 const int cb = k % kCbStages;
-                wait_bar(bars + kEmptyCB + cb, ((k / kCbStages) & 1) ^ 1, abort_flag, p.status);
-                mbar_arrive_expect_tx(bars + kFullCB + cb, 2 * kTileBytesCB);
+                const bool ready = __shfl_sync(0xffffffffu,
+                    mbar_test_wait(bars + kEmptyCB + cb, ((k / kCbStages) & 1) ^ 1) ? 1 : 0, 0) != 0;
+                if (ready) {
+                    const int g = s.h / (p.H / p.G);
+                    const int t0 = s.tile * kT;
+                    if (elect_one_sync()) {
+                        if (pf.valid) tma_prefetch_l2_4d(&tmX, 0, pf.h, pf.tile * kT, pf.b);
+                        mbar_arrive_expect_tx(bars + kFullCB + cb, 2 * kTileBytesCB);
 #pragma unroll
-                for (int q = 0; q < kN / 64; ++q) {
-                    tma_load_4d(sm + Smem::kC + cb * kTileBytesCB + q * 16384, &tmC, q * 64, g, t0,
-                                s.b, bars + kFullCB + cb);
-                    tma_load_4d(sm + Smem::kB + cb * kTileBytesCB + q * 16384, &tmB, q * 64, g, t0,
-                                s.b, bars + kFullCB + cb);
+                        for (int q = 0; q < kN / 64; ++q) {
+                            tma_load_4d(sm + Smem::kC + cb * kTileBytesCB + q * 16384, &tmC, q * 64, g,
+                                        t0, s.b, bars + kFullCB + cb);
+                            tma_load_4d(sm + Smem::kB + cb * kTileBytesCB + q * 16384, &tmB, q * 64, g,
+                                        t0, s.b, bars + kFullCB + cb);
+                        }
+                    }
+                    __syncwarp();
+                    ++k;
+                    s.next(p);
+                    if (pf.valid) pf.next(p);
+                    issued = true;
                 }
-                if (sx.valid) load_x(kx++);
             }
-            // drain: every load issued has landed before the CTA can exit
-            for (int j = max(0, k - kCbStages); j < k; ++j)
-                mbar_wait(bars + kFullCB + j % kCbStages, (j / kCbStages) & 1, kMbarLimit);
-            for (int j = max(0, kx - kXStages); j < kx; ++j)
-                mbar_wait(bars + kFullX + j % kXStages, (j / kXStages) & 1, kMbarLimit);
+            if (sx.valid) {
+                const int xs = kx % kXStages;
+                const bool ready = __shfl_sync(0xffffffffu,
+                    mbar_test_wait(bars + kEmptyX + xs, ((kx / kXStages) & 1) ^ 1) ? 1 : 0, 0) != 0;
+                if (ready) {
+                    if (elect_one_sync()) {
+                        mbar_arrive_expect_tx(bars + kFullX + xs, kTileBytesX);
+                        tma_load_4d(sm + Smem::kX + xs * kTileBytesX, &tmX, 0, sx.h, sx.tile * kT,
+                                    sx.b, bars + kFullX + xs);
+                    }
+                    __syncwarp();
+                    ++kx;
+                    sx.next(p);
+                    issued = true;
+                }
+            }
+            if (issued) {
+                idle_since = 0;
+            } else {
+                // nothing free: back off, and give up after ~2 s without progress
+                const uint64_t now = global_timer_ns();
+                if (idle_since == 0) {
+                    idle_since = now;
+                } else if (now - idle_since > 2000000000ull) {
+                    if (lane == 0) wait_gave_up(abort_flag, p.status);
+                    __syncwarp();
+                    break;
+                }
+                __nanosleep(64);
+            }
         }
+        // drain: every load issued has landed before the CTA can exit
+        for (int j = max(0, k - kCbStages); j < k; ++j)
+            mbar_wait(bars + kFullCB + j % kCbStages, (j / kCbStages) & 1, kMbarLimit);
+        for (int j = max(0, kx - kXStages); j < kx; ++j)
+            mbar_wait(bars + kFullX + j % kXStages, (j / kXStages) & 1, kMbarLimit);
     } else if (warp == kWarpMmaA) {
         // ---------------------------------------------- stream A: MMA1, states
-        if (lane == 0) {
-            constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
-            constexpr uint32_t id_st = idesc_bf16(128, kP, true, true);
-            const uint32_t xt_base = smem_addr(sm + Smem::kXt);
-            Seq s;
-            s.begin(p);
-            for (int k = 0; s.valid; ++k, s.next(p)) {
-                const int cb = k % kCbStages, sb = k & 1;
-                const uint32_t c_base = smem_addr(sm + Smem::kC + cb * kTileBytesCB);
-                const uint32_t b_base = smem_addr(sm + Smem::kB + cb * kTileBytesCB);
-                wait_bar(bars + kFullCB + cb, (k / kCbStages) & 1, abort_flag, p.status);
-                // S[sb] held S~ and Ys of tile k-2 until its epilogue read them
-                if (k >= 2) wait_bar(bars + kEmptyY + sb, ((k - 2) >> 1) & 1, abort_flag, p.status);
-                tc_fence_after_sync();
+        constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
+        constexpr uint32_t id_st = idesc_bf16(128, kP, true, true);
+        // descriptors of stage 0; a stage or K step only moves the start address
+        const uint64_t dc0 = sdesc_sw128(smem_addr(sm + Smem::kC), 16, 1024);
+        const uint64_t db0 = sdesc_sw128(smem_addr(sm + Smem::kB), 16, 1024);
+        const uint64_t dbt0 = sdesc_sw128(smem_addr(sm + Smem::kB), 16384, 1024);  // B^T, MN-major
+        const uint64_t dxt = sdesc_sw128(smem_addr(sm + Smem::kXt), 16384, 1024);
+        Seq s;
+        s.begin(p);
+        for (int k = 0; s.valid; ++k, s.next(p)) {
+            const int cb = k % kCbStages, sb = k & 1;
+            const uint64_t dc = dc0 + cb * (kTileBytesCB >> 4);
+            const uint64_t db = db0 + cb * (kTileBytesCB >> 4);
+            const uint64_t dbt = dbt0 + cb * (kTileBytesCB >> 4);
+            wait_bar(bars + kFullCB + cb, (k / kCbStages) & 1, abort_flag, p.status);
+            // S[sb] held S~ and Ys of tile k-2 until its epilogue read them
+            if (k >= 2) wait_bar(bars + kEmptyY + sb, ((k - 2) >> 1) & 1, abort_flag, p.status);
+            tc_fence_after_sync();
+            if (elect_one_sync()) {
 #pragma unroll
                 for (int q = 0; q < kN / 16; ++q) {
-                    const uint32_t off = (q >> 2) * 16384 + (q & 3) * 32;
-                    mma_bf16(tmem + kColS + sb * 128, sdesc_sw128(c_base + off, 16, 1024),
-                             sdesc_sw128(b_base + off, 16, 1024), id_s, q > 0);
+                    const uint32_t off = ((q >> 2) * 16384 + (q & 3) * 32) >> 4;
+                    mma_bf16(tmem + kColS + sb * 128, dc + off, db + off, id_s, q > 0);
                 }
                 mma_commit(bars + kFullS + sb);
-                wait_bar(bars + kEmptyStates + sb, ((k >> 1) & 1) ^ 1, abort_flag, p.status);
-                wait_bar(bars + kFullXt, k & 1, abort_flag, p.status);
-                tc_fence_after_sync();
+            }
+            __syncwarp();
+            wait_bar(bars + kEmptyStates + sb, ((k >> 1) & 1) ^ 1, abort_flag, p.status);
+            wait_bar(bars + kFullXt, k & 1, abort_flag, p.status);
+            tc_fence_after_sync();
+            if (elect_one_sync()) {
 #pragma unroll
-                for (int q = 0; q < kT / 16; ++q) {
-                    mma_bf16(tmem + kColSt + sb * 64, sdesc_sw128(b_base + q * 2048, 16384, 1024),
-                             sdesc_sw128(xt_base + q * 2048, 16384, 1024), id_st, q > 0);
-                }
+                for (int q = 0; q < kT / 16; ++q)
+                    mma_bf16(tmem + kColSt + sb * 64, dbt + q * (2048 >> 4), dxt + q * (2048 >> 4), id_st,
+                             q > 0);
                 mma_commit(bars + kEmptyXt);
                 mma_commit(bars + kFullStates + sb);
                 mma_commit(bars + kEmptyCB + cb);
             }
-            mma_commit(bars + kDrain);
-            mbar_wait(bars + kDrain, 0, kMbarLimit);
+            __syncwarp();
         }
+        if (elect_one_sync()) mma_commit(bars + kDrain);
+        __syncwarp();
+        mbar_wait(bars + kDrain, 0, kMbarLimit);
     } else if (warp == kWarpMmaB) {
         // ----------------------------------------------- stream B: MMA2, MMA3
-        if (lane == 0) {
-            constexpr uint32_t id_y2 = idesc_bf16(128, kP, false, true);
-            const uint32_t hs_base = smem_addr(sm + Smem::kHs);
-            Seq s;
-            s.begin(p);
-            for (int k = 0; s.valid; ++k, s.next(p)) {
-                const int cb = k % kCbStages, xs = k % kXStages, sb = k & 1;
-                const uint32_t c_base = smem_addr(sm + Smem::kC + cb * kTileBytesCB);
-                const uint32_t x_base = smem_addr(sm + Smem::kX + xs * kTileBytesX);
-                wait_bar(bars + kFullSt + sb, (k >> 1) & 1, abort_flag, p.status);
-                wait_bar(bars + kEmptyY + sb, ((k >> 1) & 1) ^ 1, abort_flag, p.status);
-                wait_bar(bars + kFullX + xs, (k / kXStages) & 1, abort_flag, p.status);
-                tc_fence_after_sync();
+        constexpr uint32_t id_y2 = idesc_bf16(128, kP, false, true);
+        const uint64_t dc0 = sdesc_sw128(smem_addr(sm + Smem::kC), 16, 1024);
+        const uint64_t dx0 = sdesc_sw128(smem_addr(sm + Smem::kX), 16384, 1024);
+        const uint64_t dhs = sdesc_sw128(smem_addr(sm + Smem::kHs), 16384, 1024);
+        Seq s;
+        s.begin(p);
+        for (int k = 0; s.valid; ++k, s.next(p)) {
+            const int cb = k % kCbStages, xs = k % kXStages, sb = k & 1;
+            const uint64_t dc = dc0 + cb * (kTileBytesCB >> 4);
+            const uint64_t dx = dx0 + xs * (kTileBytesX >> 4);
+            wait_bar(bars + kFullSt + sb, (k >> 1) & 1, abort_flag, p.status);
+            wait_bar(bars + kEmptyY + sb, ((k >> 1) & 1) ^ 1, abort_flag, p.status);
+            wait_bar(bars + kFullX + xs, (k / kXStages) & 1, abort_flag, p.status);
+            tc_fence_after_sync();
+            if (elect_one_sync()) {
 #pragma unroll
-                for (int q = 0; q < kT / 16; ++q) {
+                for (int q = 0; q < kT / 16; ++q)
                     mma_bf16_tmem_a(tmem + kColY + sb * 64, tmem + kColS + sb * 128 + q * 8,
-                                    sdesc_sw128(x_base + q * 2048, 16384, 1024), id_y2, q > 0);
-                }
-                wait_bar(bars + kFullCB + cb, (k / kCbStages) & 1, abort_flag, p.status);
-                wait_bar(bars + kFullHs, k & 1, abort_flag, p.status);
-                tc_fence_after_sync();
+                                    dx + q * (2048 >> 4), id_y2, q > 0);
+            }
+            __syncwarp();
+            wait_bar(bars + kFullCB + cb, (k / kCbStages) & 1, abort_flag, p.status);
+            wait_bar(bars + kFullHs, k & 1, abort_flag, p.status);
+            tc_fence_after_sync();
+            if (elect_one_sync()) {
 #pragma unroll
-                for (int q = 0; q < kN / 16; ++q) {
-                    mma_bf16(tmem + kColS + sb * 128 + 64,
-                             sdesc_sw128(c_base + (q >> 2) * 16384 + (q & 3) * 32, 16, 1024),
-                             sdesc_sw128(hs_base + q * 2048, 16384, 1024), id_y2, q > 0);
-                }
+                for (int q = 0; q < kN / 16; ++q)
+                    mma_bf16(tmem + kColS + sb * 128 + 64, dc + (((q >> 2) * 16384 + (q & 3) * 32) >> 4),
+                             dhs + q * (2048 >> 4), id_y2, q > 0);
                 mma_commit(bars + kFullY + sb);
                 mma_commit(bars + kEmptyHs);
                 mma_commit(bars + kEmptyX + xs);
                 mma_commit(bars + kEmptyCB + cb);
             }
-            mma_commit(bars + kDrain + 1);
-            mbar_wait(bars + kDrain + 1, 0, kMbarLimit);
+            __syncwarp();
         }
+        if (elect_one_sync()) mma_commit(bars + kDrain + 1);
+        __syncwarp();
+        mbar_wait(bars + kDrain + 1, 0, kMbarLimit);
     } else if (warp == kWarpPrepA || warp == kWarpPrepB) {
         // ------------------------------------- prologue: cumsum, factors, w o X
         const int wq = warp == kWarpPrepA ? 0 : 1;

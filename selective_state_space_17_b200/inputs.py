@@ -120,6 +120,13 @@ def make_inputs(Bsz, L, H, P, G, N, dtype="bf16", seed=0, kind="random") -> SSDI
     elif kind == "zero_decay":
         dt64 = np.full_like(dt64, 0.1)
         A64 = np.full_like(A64, -1.0e4)
+    elif kind == "mixed_decay":
+        # heads 1 mod 3 decay by 2^-70 .. 2^-700 per token, heads 2 mod 3 have
+        # a zero step every 37th token, the rest are drawn as above
+        strong = -np.exp(s_A.uniform(math.log(500.0), math.log(5000.0), (H,)))
+        A64 = np.where(np.arange(H) % 3 == 1, strong, A64)
+        gaps = (np.arange(L)[None, :, None] % 37 == 5) & (np.arange(H)[None, None, :] % 3 == 2)
+        dt64 = np.where(gaps, 0.0, dt64)
     elif kind != "random":
         raise ValueError(f"unknown input kind {kind!r}")
     return SSDInputs(dtype, x, dt64.astype(np.float32), A64.astype(np.float32), Bm, Cm,

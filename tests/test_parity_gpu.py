@@ -81,6 +81,14 @@ def test_special_cases(ssd, oracle, kind, dtype):
     _full_check(ssd, oracle, inp, 128 if dtype == "bf16" else 64)
 
 
+@pytest.mark.parametrize("shape", [(2, 640, 6, 64, 1, 128), (1, 300, 3, 64, 3, 128)])
+def test_tensor_core_mixed_decay(ssd, oracle, shape):
+    """Tiles whose decay or zero steps rule out the factored mask take the exact
+    form; the other tiles of the same launch take the factored one."""
+    inp = gen.make_inputs(*shape, "bf16", seed=8, kind="mixed_decay")
+    _full_check(ssd, oracle, inp, 128)
+
+
 def test_initial_state_and_no_skip_term(ssd, oracle):
     inp = gen.make_inputs(2, 384, 4, 64, 1, 128, "bf16", seed=6)
     rng = np.random.default_rng(0)
