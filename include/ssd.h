@@ -88,9 +88,11 @@ size_t ssd_workspace_size(int B, int L, int H, int P, int G, int N, int chunk, s
  *   Sizes: B, L >= 0 (B*L == 0 is a no-op apart from final_state =
  *   initial_state or 0), H >= 1, G >= 1, H % G == 0, P in [1, 256],
  *   N in [1, 256]. All pointers 16-byte aligned.
- *   The tensor-core path is taken for bf16 with P == 64, N % 16 == 0,
- *   16 <= N <= 256, chunk in {128, 256}, H % G == 0 and every row stride a
- *   multiple of 16 bytes; other valid sizes run the SIMT path.
+ *   The tensor-core path is taken for bf16 with P == 64, N a multiple of 8
+ *   with 8 <= N <= 128, and chunk in {64, 128, 256}; other valid sizes run
+ *   the SIMT path. The tensor-core path evaluates the chunked form on
+ *   128-token tiles whatever `chunk` is (the result does not depend on the
+ *   chunk length beyond rounding).
  */
 ssd_status ssd_forward(const void* x, const float* dt, const float* A, const void* Bm,
                        const void* Cm, const float* D, const float* initial_state, void* y,
@@ -103,12 +105,12 @@ ssd_status ssd_forward(const void* x, const float* dt, const float* A, const voi
  * device memory. The pages describe no such entry point; it is a convenience
  * of this library. It takes the same arguments as ssd_forward without the
  * workspace: its scratch (look-back control words and the per-head state
- * ring, 256 + 4*B*H rounded to 256 + 2*B*H*P*N*4 bytes) lives in a fixed
+ * ring, 256 + 4*B*H rounded to 256 + 2*B*H*64*128*4 bytes) lives in a fixed
  * 24 MiB device array inside the library, which every GPU that loads the
  * library holds until the process exits. Only the tensor-core sizes are
- * handled (bf16, P == 64, N == 128, chunk 128 or 256, B*L > 0); other sizes
- * return SSD_ERR_UNSUPPORTED, and sizes whose scratch exceeds the array
- * (B*H > 383 at N == 128) return SSD_ERR_WORKSPACE before anything is
+ * handled (bf16, P == 64, N a multiple of 8 up to 128, chunk 64, 128 or 256,
+ * B*L > 0); other sizes return SSD_ERR_UNSUPPORTED, and sizes whose scratch
+ * exceeds the array (B*H > 383) return SSD_ERR_WORKSPACE before anything is
  * enqueued. The call allocates nothing. The first call on each device looks
  * up the array's device address (make it before any stream capture). All
  * calls on a device share the array: calls that may overlap on the GPU race

@@ -71,7 +71,7 @@ using namespace sm100;
 
 constexpr int kT = 128;   // tokens per tile
 constexpr int kP = 64;    // head dim on this path
-constexpr int kN = 128;   // state dim on this path
+constexpr int kN = 128;   // state dim of the tiles; a smaller N is zero-padded up to it
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint64_t kMbarLimit = 1ull << 22;  // polls; each wait is also capped at ~2 s
 
@@ -114,6 +114,8 @@ struct TcParams {
     unsigned int* status;
     unsigned long long wait_limit;
     int B, L, H, G;
+    int N;        // state dim (<= kN)
+    int nkh;      // 64-wide halves of the state dim that hold data (1 or 2)
     int ntiles;   // tiles per chain
     int chains;   // B * H
     int seg_len;  // tiles per segment
@@ -267,6 +269,17 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         tmem_alloc(s_tmem, kTmemCols);
         tmem_relinquish();
     }
+    if (p.nkh == 1) {
+        // N <= 64: the second half of every C/B tile is never loaded; zero it
+        // once so the states MMA (which spans the full 128 rows) reads zeros
+        for (int cb = 0; cb < kCbStages; ++cb)
+            for (int base = 0; base < 2; ++base) {
+                uint4* z = reinterpret_cast<uint4*>(sm + (base ? Smem::kB : Smem::kC) +
+                                                    cb * kTileBytesCB + 16384);
+                for (int u = tid; u < 16384 / 16; u += kThreads) z[u] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        fence_async_shared();
+    }
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
@@ -297,9 +310,10 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     const int t0 = s.tile * kT;
                     if (elect_one_sync()) {
                         if (pf.valid) tma_prefetch_l2_4d(&tmX, 0, pf.h, pf.tile * kT, pf.b);
-                        mbar_arrive_expect_tx(bars + kFullCB + cb, 2 * kTileBytesCB);
+                        mbar_arrive_expect_tx(bars + kFullCB + cb, p.nkh * 2 * 16384);
 #pragma unroll
                         for (int q = 0; q < kN / 64; ++q) {
+                            if (q >= p.nkh) break;
                             tma_load_4d(sm + Smem::kC + cb * kTileBytesCB + q * 16384, &tmC, q * 64, g,
                                         t0, s.b, bars + kFullCB + cb);
                             tma_load_4d(sm + Smem::kB + cb * kTileBytesCB + q * 16384, &tmB, q * 64, g,
@@ -372,6 +386,7 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             if (elect_one_sync()) {
 #pragma unroll
                 for (int q = 0; q < kN / 16; ++q) {
+                    if (q >= 4 * p.nkh) break;
                     const uint32_t off = ((q >> 2) * 16384 + (q & 3) * 32) >> 4;
                     mma_bf16(tmem + kColS + sb * 128, dc + off, db + off, id_s, q > 0);
                 }
@@ -423,9 +438,11 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             tc_fence_after_sync();
             if (elect_one_sync()) {
 #pragma unroll
-                for (int q = 0; q < kN / 16; ++q)
+                for (int q = 0; q < kN / 16; ++q) {
+                    if (q >= 4 * p.nkh) break;
                     mma_bf16(tmem + kColS + sb * 128 + 64, dc + (((q >> 2) * 16384 + (q & 3) * 32) >> 4),
                              dhs + q * (2048 >> 4), id_y2, q > 0);
+                }
                 mma_commit(bars + kFullY + sb);
                 mma_commit(bars + kEmptyHs);
                 mma_commit(bars + kEmptyX + xs);
@@ -601,7 +618,8 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         const int wq = warp - kWgOut0;
         const int n = wq * 32 + lane;  // state row / tile row / TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-        const size_t PN = static_cast<size_t>(kP) * kN;
+        const size_t PN = static_cast<size_t>(kP) * p.N;
+        const bool n_live = n < p.N;  // rows past N are zero padding
         float h[kP];
         // the bf16 h_prev operand of MMA3 for tile kk (row n of [N][P],
         // MN-major), once MMA3 of tile kk - 1 has read the previous one
@@ -631,7 +649,8 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 if (s.seg == 0) {
                     const float* src = p.init ? p.init + static_cast<size_t>(s.chain) * PN : nullptr;
 #pragma unroll
-                    for (int q = 0; q < kP; ++q) h[q] = src ? src[static_cast<size_t>(q) * kN + n] : 0.f;
+                    for (int q = 0; q < kP; ++q)
+                        h[q] = src && n_live ? src[static_cast<size_t>(q) * p.N + n] : 0.f;
                 } else {
                     if (n == 0 && !*abort_flag) {
                         const unsigned int* f = p.flags + s.chain;
@@ -688,8 +707,10 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 if (s.tile == p.ntiles - 1) {
                     if (p.final_state) {
                         float* dst = p.final_state + static_cast<size_t>(s.chain) * PN;
+                        if (n_live) {
 #pragma unroll
-                        for (int q = 0; q < kP; ++q) dst[static_cast<size_t>(q) * kN + n] = h[q];
+                            for (int q = 0; q < kP; ++q) dst[static_cast<size_t>(q) * p.N + n] = h[q];
+                        }
                     }
                 } else {
                     float4* dst = reinterpret_cast<float4*>(
@@ -809,7 +830,7 @@ WsLayout ws_layout(const FwdArgs& a)
     w.ctrl = 0;
     w.flags = 256;
     w.ring = w.flags + ((chains * 4 + 255) / 256) * 256;
-    w.total = w.ring + chains * 2 * kP * a.N * sizeof(float);
+    w.total = w.ring + chains * 2 * kP * kN * sizeof(float);
     return w;
 }
 
@@ -828,8 +849,8 @@ void choose_segments(int ntiles, int chains, int ctas, int* seg_len, int* nseg)
 cudaError_t launch(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)
 {
     CUtensorMap tmX, tmB, tmC, tmY;
-    if (!make_map(&tmX, a.x, kP, a.H, a.L, a.B) || !make_map(&tmB, a.Bm, kN, a.G, a.L, a.B) ||
-        !make_map(&tmC, a.Cm, kN, a.G, a.L, a.B) || !make_map(&tmY, a.y, kP, a.H, a.L, a.B))
+    if (!make_map(&tmX, a.x, kP, a.H, a.L, a.B) || !make_map(&tmB, a.Bm, a.N, a.G, a.L, a.B) ||
+        !make_map(&tmC, a.Cm, a.N, a.G, a.L, a.B) || !make_map(&tmY, a.y, kP, a.H, a.L, a.B))
         return cudaErrorInvalidValue;
     const WsLayout w = ws_layout(a);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -849,6 +870,8 @@ cudaError_t launch(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)
     p.L = a.L;
     p.H = a.H;
     p.G = a.G;
+    p.N = a.N;
+    p.nkh = a.N <= 64 ? 1 : 2;
     p.ntiles = (a.L + kT - 1) / kT;
     p.chains = a.B * a.H;
     const int ctas_max = ctx.num_sms > 0 ? ctx.num_sms : 1;
@@ -868,7 +891,8 @@ cudaError_t launch(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)
 
 bool tc_supported(const FwdArgs& a)
 {
-    return a.bf16 && a.P == kP && a.N == kN && (a.chunk == 128 || a.chunk == 256) &&
+    return a.bf16 && a.P == kP && a.N % 8 == 0 && a.N >= 8 && a.N <= kN &&
+           (a.chunk == 64 || a.chunk == 128 || a.chunk == 256) &&
            static_cast<long long>(a.B) * a.L > 0 &&
            static_cast<long long>((a.L + kT - 1) / kT) * a.B * a.H < (1ll << 31);
 }

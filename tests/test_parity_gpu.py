@@ -81,6 +81,17 @@ def test_special_cases(ssd, oracle, kind, dtype):
     _full_check(ssd, oracle, inp, 128 if dtype == "bf16" else 64)
 
 
+@pytest.mark.parametrize("N,chunk", [(8, 64), (48, 128), (64, 256), (96, 64), (120, 128)])
+def test_tensor_core_state_dims(ssd, oracle, N, chunk):
+    """State dims below 128 run on the tensor-core path with the state rows
+    zero-padded to 128 (a ragged tail, an initial state and two groups too)."""
+    inp = gen.make_inputs(2, 300, 4, 64, 2, N, "bf16", seed=9)
+    rng = np.random.default_rng(1)
+    init = rng.standard_normal((2, 4, 64, N)).astype(np.float32)
+    assert ssd.kernel_count(2, 300, 4, 64, 2, N, chunk, 1) == 1
+    _full_check(ssd, oracle, inp, chunk, init=init)
+
+
 @pytest.mark.parametrize("shape", [(2, 640, 6, 64, 1, 128), (1, 300, 3, 64, 3, 128)])
 def test_tensor_core_mixed_decay(ssd, oracle, shape):
     """Tiles whose decay or zero steps rule out the factored mask take the exact

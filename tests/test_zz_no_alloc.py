@@ -69,11 +69,11 @@ def test_noalloc_refuses_what_it_cannot_run(ssd):
     y = torch.empty_like(t["x"])
     fs = torch.empty((8, 64, 64, 128), dtype=torch.float32, device="cuda")
     assert _noalloc(ssd, t, y, fs, big, 128, stream) == 6  # SSD_ERR_WORKSPACE
-    # N = 64 is not a tensor-core size
-    small = (1, 256, 2, 64, 1, 64)
+    # N = 256 is not a tensor-core size (the tiles hold N <= 128)
+    small = (1, 256, 2, 64, 1, 256)
     t = to_device(gen.make_inputs(*small, "bf16", seed=34))
     y = torch.empty_like(t["x"])
-    fs = torch.empty((1, 2, 64, 64), dtype=torch.float32, device="cuda")
+    fs = torch.empty((1, 2, 64, 256), dtype=torch.float32, device="cuda")
     assert _noalloc(ssd, t, y, fs, small, 128, stream) == 2  # SSD_ERR_UNSUPPORTED
     torch.cuda.synchronize()
     assert np.isfinite(to_host_f64(t["x"][:1, :1])).all()
