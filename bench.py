@@ -36,6 +36,10 @@ from selective_state_space_17_b200 import inputs as gen  # noqa: E402
 METRIC = "SSD fwd Mtokens/s per layer on 1 B200; % of HBM/tensor-core roofline"
 UNIT = "Mtokens/s"
 WORKLOAD = gen.LAYER_2P7B
+# other configurations of the same layer, selectable with --workload (the
+# default is the one the metric is quoted on)
+WORKLOADS = {"2.7b": gen.LAYER_2P7B, "370m": gen.LAYER_370M, "long": gen.LONG_CONTEXT}
+WORKLOADS.update({f"sweep-n{w.N}-q{w.chunk}": w for w in gen.sweep_workloads()})
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -186,7 +190,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    w = WORKLOAD
+    w = args.workload
     inp = w.make(0)
     per_step = []
     info = None
@@ -236,7 +240,7 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize()
 
-    w = WORKLOAD
+    w = args.workload
     inp = w.make(seed=rank)
     code = ssd.SSD_BF16 if w.dtype == "bf16" else ssd.SSD_F32
 
@@ -417,7 +421,10 @@ def main():
                     help="skip the oracle timing on the host cores")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer end-to-end timing (used for profiling runs)")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="2.7b",
+                    help="layer configuration (default: the 2.7B-shaped layer)")
     args = ap.parse_args()
+    args.workload = WORKLOADS[args.workload]
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps, reported as run
     if args.impl == "reference":
         return run_reference(args)
