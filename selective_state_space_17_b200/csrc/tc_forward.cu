@@ -111,6 +111,15 @@ struct TcParams {
     unsigned int* ctrl;   // [1] CTAs done
     unsigned int* flags;  // per chain: number of segments published
     float* ring;          // per chain: 2 slots of [N][P] fp32
+    // Segment-parallel form (chains with many segments): `mode` 1 computes each
+    // segment's local end state from zero and its total log2 decay (no y, no
+    // look-back); mode 2 starts each segment from the state that a scan over
+    // those wrote to seg_hin (no look-back, no publication); mode 0 is the
+    // single pass with look-back.
+    int mode;
+    float* seg_state;     // [chain][seg][kN][kP]
+    float* seg_decay;     // [chain][seg]
+    const float* seg_hin; // [chain][seg][kN][kP]
     unsigned int* status;
     unsigned long long wait_limit;
     int B, L, H, G;
@@ -621,6 +630,7 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         const size_t PN = static_cast<size_t>(kP) * p.N;
         const bool n_live = n < p.N;  // rows past N are zero padding
         float h[kP];
+        float lam = 0.f;  // log2 decay of the segment so far (mode 1)
         // the bf16 h_prev operand of MMA3 for tile kk (row n of [N][P],
         // MN-major), once MMA3 of tile kk - 1 has read the previous one
         auto write_hs = [&](int kk) {
@@ -645,33 +655,44 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             const bool last = s.tile == s.tile_end - 1;
             const int c = k % kCsStages, sb = k & 1;
             if (first) {
-                // look-back: the state before this segment
-                if (s.seg == 0) {
-                    const float* src = p.init ? p.init + static_cast<size_t>(s.chain) * PN : nullptr;
+                // the state entering this segment: zero (a segment's local state,
+                // mode 1), the initial state (first segment), or the state the
+                // predecessor published (mode 0, after a bounded acquire poll) or
+                // the scan wrote (mode 2)
+                lam = 0.f;
+                if (p.mode == 1 || (s.seg == 0 && !p.init)) {
 #pragma unroll
-                    for (int q = 0; q < kP; ++q)
-                        h[q] = src && n_live ? src[static_cast<size_t>(q) * p.N + n] : 0.f;
+                    for (int q = 0; q < kP; ++q) h[q] = 0.f;
+                } else if (s.seg == 0) {
+                    const float* src = p.init + static_cast<size_t>(s.chain) * PN;
+#pragma unroll
+                    for (int q = 0; q < kP; ++q) h[q] = n_live ? src[static_cast<size_t>(q) * p.N + n] : 0.f;
                 } else {
-                    if (n == 0 && !*abort_flag) {
-                        const unsigned int* f = p.flags + s.chain;
-                        bool ok = false;
-                        const uint64_t t0 = global_timer_ns();
-                        for (unsigned long long it = 0; it < p.wait_limit; ++it) {
-                            if (ld_acquire_gpu(f) >= static_cast<unsigned int>(s.seg)) {
-                                ok = true;
-                                break;
+                    if (p.mode == 0) {
+                        if (n == 0 && !*abort_flag) {
+                            const unsigned int* f = p.flags + s.chain;
+                            bool ok = false;
+                            const uint64_t t0 = global_timer_ns();
+                            for (unsigned long long it = 0; it < p.wait_limit; ++it) {
+                                if (ld_acquire_gpu(f) >= static_cast<unsigned int>(s.seg)) {
+                                    ok = true;
+                                    break;
+                                }
+                                if ((it & 255) == 255 && global_timer_ns() - t0 > 4000000000ull) break;
+                                __nanosleep(64);
                             }
-                            if ((it & 255) == 255 && global_timer_ns() - t0 > 4000000000ull) break;
-                            __nanosleep(64);
+                            if (!ok) {
+                                record_status(p.status, kDevWaitTimeout);
+                                *abort_flag = 1;
+                            }
                         }
-                        if (!ok) {
-                            record_status(p.status, kDevWaitTimeout);
-                            *abort_flag = 1;
-                        }
+                        named_bar_sync(kBarOut, 128);
                     }
-                    named_bar_sync(kBarOut, 128);
+                    const size_t slot = p.mode == 2
+                                            ? static_cast<size_t>(s.chain) * p.nseg + s.seg
+                                            : static_cast<size_t>(s.chain) * 2 + ((s.seg - 1) & 1);
                     const float4* src = reinterpret_cast<const float4*>(
-                        p.ring + ((static_cast<size_t>(s.chain) * 2 + ((s.seg - 1) & 1)) * kN + n) * kP);
+                        (p.mode == 2 ? p.seg_hin : p.ring) + (slot * kN + n) * kP);
 #pragma unroll
                     for (int q = 0; q < kP / 4; ++q) {
                         const float4 v = __ldcg(src + q);
@@ -703,25 +724,32 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             named_bar_sync(kBarOut, 128);
             if (n == 0) mbar_arrive(bars + kEmptyStates + sb);
 
+            if (p.mode == 1) lam += r.cs[kT - 1];
             if (last) {
                 if (s.tile == p.ntiles - 1) {
-                    if (p.final_state) {
+                    if (p.final_state && n_live) {
                         float* dst = p.final_state + static_cast<size_t>(s.chain) * PN;
-                        if (n_live) {
 #pragma unroll
-                            for (int q = 0; q < kP; ++q) dst[static_cast<size_t>(q) * p.N + n] = h[q];
-                        }
+                        for (int q = 0; q < kP; ++q) dst[static_cast<size_t>(q) * p.N + n] = h[q];
                     }
-                } else {
-                    float4* dst = reinterpret_cast<float4*>(
-                        p.ring + ((static_cast<size_t>(s.chain) * 2 + (s.seg & 1)) * kN + n) * kP);
+                } else if (p.mode != 2) {
+                    // mode 0 publishes the segment's end state to the ring; mode 1
+                    // stores the local end state and the segment's decay
+                    const size_t slot = p.mode == 1 ? static_cast<size_t>(s.chain) * p.nseg + s.seg
+                                                    : static_cast<size_t>(s.chain) * 2 + (s.seg & 1);
+                    float4* dst = reinterpret_cast<float4*>((p.mode == 1 ? p.seg_state : p.ring) +
+                                                            (slot * kN + n) * kP);
 #pragma unroll
                     for (int q = 0; q < kP / 4; ++q)
                         dst[q] = make_float4(h[q * 4], h[q * 4 + 1], h[q * 4 + 2], h[q * 4 + 3]);
-                    __threadfence();
-                    named_bar_sync(kBarOut, 128);
-                    if (n == 0 && !p.skip_publish)
-                        st_release_gpu(p.flags + s.chain, static_cast<unsigned int>(s.seg + 1));
+                    if (p.mode == 1) {
+                        if (n == 0) p.seg_decay[slot] = lam;
+                    } else {
+                        __threadfence();
+                        named_bar_sync(kBarOut, 128);
+                        if (n == 0 && !p.skip_publish)
+                            st_release_gpu(p.flags + s.chain, static_cast<unsigned int>(s.seg + 1));
+                    }
                 }
             }
 
@@ -759,8 +787,10 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             tc_fence_before_sync();
             named_bar_sync(kBarOut, 128);
             if (n == 0) {
-                tma_store_4d(&tmY, sm + Smem::kYs, 0, s.h, s.tile * kT, s.b);
-                tma_store_commit();
+                if (p.mode != 1) {
+                    tma_store_4d(&tmY, sm + Smem::kYs, 0, s.h, s.tile * kT, s.b);
+                    tma_store_commit();
+                }
                 mbar_arrive(bars + kEmptyY + sb);
                 mbar_arrive(bars + kEmptyRec + c);
             }
@@ -819,23 +849,6 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint
     return r == CUDA_SUCCESS;
 }
 
-struct WsLayout {
-    size_t ctrl, flags, ring, total;
-};
-
-WsLayout ws_layout(const FwdArgs& a)
-{
-    WsLayout w;
-    const size_t chains = static_cast<size_t>(a.B) * a.H;
-    w.ctrl = 0;
-    w.flags = 256;
-    w.ring = w.flags + ((chains * 4 + 255) / 256) * 256;
-    w.total = w.ring + chains * 2 * kP * kN * sizeof(float);
-    return w;
-}
-
-int g_skip_publish = 0;
-
 // Segments per chain: enough items for about eight per CTA, at least one tile each.
 void choose_segments(int ntiles, int chains, int ctas, int* seg_len, int* nseg)
 {
@@ -846,13 +859,97 @@ void choose_segments(int ntiles, int chains, int ctas, int* seg_len, int* nseg)
     *nseg = (ntiles + *seg_len - 1) / *seg_len;
 }
 
+// Chains cut into this many segments or more run segment-parallel (three
+// launches) instead of waiting on each other's published states one after
+// another.
+constexpr int kParallelSegments = 8;
+
+int sm_count()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        return 148;
+    }
+    return n;
+}
+
+struct Segments {
+    int ntiles, chains, seg_len, nseg;
+    bool parallel;
+};
+
+Segments segments(const FwdArgs& a, int ctas)
+{
+    Segments g;
+    g.ntiles = (a.L + kT - 1) / kT;
+    g.chains = a.B * a.H;
+    choose_segments(g.ntiles, g.chains, ctas, &g.seg_len, &g.nseg);
+    g.parallel = g.nseg >= kParallelSegments;
+    return g;
+}
+
+struct WsLayout {
+    size_t ctrl, flags, ring, seg_state, seg_decay, seg_hin, total;
+};
+
+WsLayout ws_layout(const FwdArgs& a, const Segments& g)
+{
+    WsLayout w;
+    const size_t chains = static_cast<size_t>(a.B) * a.H;
+    const size_t slot = static_cast<size_t>(kP) * kN * sizeof(float);
+    w.ctrl = 0;
+    w.flags = 256;
+    w.ring = w.flags + ((chains * 4 + 255) / 256) * 256;
+    w.total = w.ring + chains * 2 * slot;
+    w.seg_state = w.seg_decay = w.seg_hin = w.total;
+    if (g.parallel) {
+        const size_t units = chains * g.nseg;
+        w.seg_state = w.total;
+        w.seg_decay = w.seg_state + units * slot;
+        w.seg_hin = w.seg_decay + ((units * 4 + 255) / 256) * 256;
+        w.total = w.seg_hin + units * slot;
+    }
+    return w;
+}
+
+int g_skip_publish = 0;
+
+// The state entering every segment of a chain, from the segments' local end
+// states and decays: h_in(0) = initial state, h_in(s + 1) = 2^decay(s) h_in(s)
+// + local(s) (the composition of affine maps of "Selective SSM guide", eq. (3),
+// applied segment by segment). One thread per state element of a chain
+// (blockIdx.y = chain); states are [kN][kP] with rows past N zero.
+constexpr int kScanThreads = 256;
+static_assert(kN * kP % kScanThreads == 0, "scan grid covers the state exactly");
+
+__global__ void __launch_bounds__(kScanThreads)
+segment_scan_kernel(const float* init, const float* seg_state, const float* seg_decay,
+                    float* seg_hin, int P, int N, int nseg)
+{
+    const size_t chain = blockIdx.y;
+    const int e = blockIdx.x * kScanThreads + threadIdx.x;  // < kN * kP by the grid
+    const int n = e / kP, q = e - n * kP;
+    float v = init && n < N ? init[(chain * P + q) * N + n] : 0.f;
+    const size_t u0 = chain * nseg;
+#pragma unroll 8
+    for (int sg = 0; sg < nseg; ++sg) {
+        seg_hin[(u0 + sg) * kN * kP + e] = v;
+        if (sg + 1 < nseg)
+            v = fmaf(exp2f(__ldg(seg_decay + u0 + sg)), v, __ldcg(seg_state + (u0 + sg) * kN * kP + e));
+    }
+}
+
 cudaError_t launch(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)
 {
     CUtensorMap tmX, tmB, tmC, tmY;
     if (!make_map(&tmX, a.x, kP, a.H, a.L, a.B) || !make_map(&tmB, a.Bm, a.N, a.G, a.L, a.B) ||
         !make_map(&tmC, a.Cm, a.N, a.G, a.L, a.B) || !make_map(&tmY, a.y, kP, a.H, a.L, a.B))
         return cudaErrorInvalidValue;
-    const WsLayout w = ws_layout(a);
+    const int ctas_max = ctx.num_sms > 0 ? ctx.num_sms : 1;
+    const Segments g = segments(a, ctas_max);
+    const WsLayout w = ws_layout(a, g);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     TcParams p;
     p.dt = a.dt;
@@ -864,6 +961,9 @@ cudaError_t launch(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)
     p.ctrl = reinterpret_cast<unsigned int*>(ws + w.ctrl);
     p.flags = reinterpret_cast<unsigned int*>(ws + w.flags);
     p.ring = reinterpret_cast<float*>(ws + w.ring);
+    p.seg_state = reinterpret_cast<float*>(ws + w.seg_state);
+    p.seg_decay = reinterpret_cast<float*>(ws + w.seg_decay);
+    p.seg_hin = reinterpret_cast<const float*>(ws + w.seg_hin);
     p.status = ctx.status;
     p.wait_limit = ctx.wait_limit;
     p.B = a.B;
@@ -872,19 +972,30 @@ cudaError_t launch(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)
     p.G = a.G;
     p.N = a.N;
     p.nkh = a.N <= 64 ? 1 : 2;
-    p.ntiles = (a.L + kT - 1) / kT;
-    p.chains = a.B * a.H;
-    const int ctas_max = ctx.num_sms > 0 ? ctx.num_sms : 1;
-    choose_segments(p.ntiles, p.chains, ctas_max, &p.seg_len, &p.nseg);
-    p.items = p.chains * p.nseg;
+    p.ntiles = g.ntiles;
+    p.chains = g.chains;
+    p.seg_len = g.seg_len;
+    p.nseg = g.nseg;
     p.skip_publish = g_skip_publish;
-    const int grid = p.items < ctas_max ? p.items : ctas_max;
     const uint32_t smem = Smem::kBytes;
     cudaError_t e = cudaFuncSetAttribute(tc_forward_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    tc_forward_kernel<<<grid, kThreads, smem, ctx.stream>>>(tmX, tmB, tmC, tmY, p);
-    return cudaGetLastError();
+    auto run = [&](int mode, int items) {
+        p.mode = mode;
+        p.items = items;
+        const int grid = items < ctas_max ? items : ctas_max;
+        tc_forward_kernel<<<grid, kThreads, smem, ctx.stream>>>(tmX, tmB, tmC, tmY, p);
+        return cudaGetLastError();
+    };
+    if (!g.parallel) return run(0, g.chains * g.nseg);
+    // segment-parallel: local states of every segment but each chain's last
+    // (segment-major numbering puts those first), the scan, then the outputs
+    if ((e = run(1, g.chains * (g.nseg - 1))) != cudaSuccess) return e;
+    segment_scan_kernel<<<dim3(kN * kP / kScanThreads, g.chains), kScanThreads, 0, ctx.stream>>>(
+        a.init, p.seg_state, p.seg_decay, reinterpret_cast<float*>(ws + w.seg_hin), kP, a.N, g.nseg);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    return run(2, g.chains * g.nseg);
 }
 
 }  // namespace
@@ -897,9 +1008,9 @@ bool tc_supported(const FwdArgs& a)
            static_cast<long long>((a.L + kT - 1) / kT) * a.B * a.H < (1ll << 31);
 }
 
-size_t tc_workspace_bytes(const FwdArgs& a) { return ws_layout(a).total; }
+size_t tc_workspace_bytes(const FwdArgs& a) { return ws_layout(a, segments(a, sm_count())).total; }
 
-int tc_kernel_count(const FwdArgs&) { return 1; }
+int tc_kernel_count(const FwdArgs& a) { return segments(a, sm_count()).parallel ? 3 : 1; }
 
 void tc_set_skip_publish(int v) { g_skip_publish = v; }
 
@@ -967,7 +1078,7 @@ extern "C" ssd_status ssd_forward_noalloc(const void* x, const float* dt, const 
     a.B = B; a.L = L; a.H = H; a.P = P; a.G = G; a.N = N; a.chunk = chunk;
     a.bf16 = dtype == SSD_BF16;
     if (!tc_supported(a)) return SSD_ERR_UNSUPPORTED;  // tensor-core sizes only
-    const WsLayout w = ws_layout(a);
+    const WsLayout w = ws_layout(a, segments(a, sm_count()));
     if (w.total > kNoAllocScratchBytes) return SSD_ERR_WORKSPACE;  // scratch would not fit
 
     int dev = 0;

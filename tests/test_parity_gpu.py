@@ -92,6 +92,22 @@ def test_tensor_core_state_dims(ssd, oracle, N, chunk):
     _full_check(ssd, oracle, inp, chunk, init=init)
 
 
+@pytest.mark.parametrize("shape,chunk,with_init", [
+    ((1, 4096, 4, 64, 1, 128), 256, False),   # 4 chains of 32 tiles: one tile per segment
+    ((2, 3000, 2, 64, 1, 64), 128, True),     # ragged tail, N = 64, initial state
+])
+def test_segment_parallel_form(ssd, oracle, shape, chunk, with_init):
+    """Few chains with many tiles: each segment's local state, a scan over the
+    segments, then the outputs (three launches instead of a serial look-back)."""
+    assert ssd.kernel_count(*shape, chunk, 1) == 3
+    inp = gen.make_inputs(*shape, "bf16", seed=10)
+    init = None
+    if with_init:
+        B, _, H, P, _, N = shape
+        init = np.random.default_rng(2).standard_normal((B, H, P, N)).astype(np.float32)
+    _full_check(ssd, oracle, inp, chunk, init=init)
+
+
 @pytest.mark.parametrize("shape", [(2, 640, 6, 64, 1, 128), (1, 300, 3, 64, 3, 128)])
 def test_tensor_core_mixed_decay(ssd, oracle, shape):
     """Tiles whose decay or zero steps rule out the factored mask take the exact
