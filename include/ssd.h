@@ -67,10 +67,13 @@ typedef enum {
 const char* ssd_status_string(ssd_status status);
 
 /* Bytes of device workspace ssd_forward needs for these sizes (0 if the sizes
- * are invalid). The workspace must be zero-filled once before its first use
- * (e.g. cudaMemset); every call leaves its control words zeroed again, so a
- * workspace can be reused by later calls on the same stream without clearing.
- * Two calls that run concurrently must not share one workspace. */
+ * are invalid). On the tensor-core path the size depends on the current
+ * device's SM count, which decides how each (batch, head) chain is cut into
+ * segments; ask on the device that will run the call. The workspace must be
+ * zero-filled once before its first use (e.g. cudaMemset); every call leaves
+ * its control words zeroed again, so a workspace can be reused by later calls
+ * on the same stream without clearing. Two calls that run concurrently must
+ * not share one workspace. */
 size_t ssd_workspace_size(int B, int L, int H, int P, int G, int N, int chunk, ssd_dtype dtype);
 
 /*
@@ -148,7 +151,11 @@ ssd_status ssd_step(const void* x, const float* dt, const float* A, const void* 
                     int P, int G, int N, ssd_dtype dtype, ssd_stream_t stream);
 
 /* Number of kernels one ssd_forward call with these sizes enqueues (0 if the
- * sizes are invalid or there are no tokens). Host-side query; no CUDA call. */
+ * sizes are invalid or there are no tokens): 1 on the tensor-core path; 3 when
+ * its chains are cut into eight or more segments (few (batch, head) chains on
+ * long sequences: every segment's local state, a scan over the segments, then
+ * the outputs); 3 on the SIMT path. Host-side query; it reads the current
+ * device's SM count and launches nothing. */
 int ssd_forward_kernel_count(int B, int L, int H, int P, int G, int N, int chunk,
                              ssd_dtype dtype);
 
