@@ -11,7 +11,8 @@ Prints one JSON line on rank 0. ``value`` is Mtokens/s over all ranks (tokens
 = B*L per rank per step; every rank runs its own copy of the layer: the work
 shards by batch and head with no data-path collective, so scaling is weak).
 Timing: CUDA events on the launching stream around each step, L2 flushed
-(256 MiB write) between steps outside the events, max over ranks.
+between steps outside the events (a 256 MiB write, then a 256 MiB read so that
+no dirty line is written back inside the next step), max over ranks.
 ``--impl reference`` times the fp64 CPU oracle on the host cores instead
 (rank 0 only), on a bounded sample of the same workload.
 """
@@ -41,6 +42,23 @@ WORKLOAD = gen.LAYER_2P7B
 WORKLOADS = {"2.7b": gen.LAYER_2P7B, "370m": gen.LAYER_370M, "long": gen.LONG_CONTEXT}
 WORKLOADS.update({f"sweep-n{w.N}-q{w.chunk}": w for w in gen.sweep_workloads()})
 L2_FLUSH_BYTES = 256 << 20
+
+
+class L2Flush:
+    """Leaves the L2 cold and clean between timed steps: a write of a buffer
+    larger than the L2 evicts everything, and a read of a second such buffer
+    then evicts the written (dirty) lines, so their write-back happens here
+    instead of inside the next timed step."""
+
+    def __init__(self, dev, nbytes=L2_FLUSH_BYTES):
+        import torch
+        self.w = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        self.r = torch.ones(nbytes, dtype=torch.uint8, device=dev)
+
+    def __call__(self):
+        import torch
+        self.w.zero_()
+        torch.sum(self.r, dtype=torch.int64)
 
 
 def compulsory_bytes(w: gen.Workload) -> int:
@@ -256,7 +274,7 @@ def run_ours(args):
     fs = torch.empty((w.B, w.H, w.P, w.N), dtype=torch.float32, device=dev)
     ws = torch.zeros(ssd.workspace_size(w.B, w.L, w.H, w.P, w.G, w.N, w.chunk, code),
                      dtype=torch.uint8, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream()
 
     def step():
@@ -264,7 +282,7 @@ def run_ours(args):
                     final_state=fs, workspace=ws, stream=stream)
 
     for _ in range(args.warmup):
-        flush.zero_()
+        flush()
         step()
     ssd.poll_status(stream)
     barrier()
@@ -273,7 +291,7 @@ def run_ours(args):
     with ClockSampler(local_rank) as clk:
         barrier()
         for i in range(args.steps):
-            flush.zero_()
+            flush()
             starts[i].record(stream)
             step()
             ends[i].record(stream)
@@ -326,11 +344,11 @@ def time_decode(ssd, dev, flush, warmup, steps, world, dist):
     y = torch.empty_like(x)
     stream = torch.cuda.current_stream()
     for _ in range(warmup):
-        flush.zero_()
+        flush()
         ssd.step(x, dt, A, Bm, Cm, D, state, y=y, stream=stream)
     times = []
     for _ in range(steps):
-        flush.zero_()
+        flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         ssd.step(x, dt, A, Bm, Cm, D, state, y=y, stream=stream)
@@ -375,7 +393,7 @@ def _report(args, w, rank, world, ms, per_step_ms, clk, inp, e2e_ms, host, ssd, 
             "config": {"workload": w.name, "global_batch": w.B * world, "seq_len": w.L,
                        "heads": w.H, "headdim": w.P, "d_state": w.N, "groups": w.G,
                        "chunk": w.chunk, "parallelism": f"replicas x{world} (batch/head shards)",
-                       "l2": "flushed between steps (256 MiB write, outside the events)"},
+                       "l2": "flushed between steps (256 MiB write, then 256 MiB read, outside the events)"},
             "roofline": {"bound": bound, "achieved": achieved_gbs if bound == "hbm" else achieved_tflops,
                          "peak": hbm_peak if bound == "hbm" else tc_peak,
                          "unit": "GB/s" if bound == "hbm" else "TFLOP/s",

@@ -112,10 +112,10 @@ struct TcParams {
     unsigned int* flags;  // per chain: number of segments published
     float* ring;          // per chain: 2 slots of [N][P] fp32
     // Segment-parallel form (chains with many segments): `mode` 1 computes each
-    // segment's local end state from zero and its total log2 decay (no y, no
-    // look-back); mode 2 starts each segment from the state that a scan over
-    // those wrote to seg_hin (no look-back, no publication); mode 0 is the
-    // single pass with look-back.
+    // segment's local end state from zero and its total log2 decay, running only
+    // the state path (B and X loads, w o X, the tile states, h); mode 2 starts
+    // each segment from the state that a scan over those wrote to seg_hin (no
+    // look-back, no publication); mode 0 is the single pass with look-back.
     int mode;
     float* seg_state;     // [chain][seg][kN][kP]
     float* seg_decay;     // [chain][seg]
@@ -260,6 +260,8 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
+    // mode 1 needs only the tile states: no C, no MMA1 / mask / MMA2 / MMA3, no y
+    const bool states_only = p.mode == 1;
 
     if (tid == 0) {
         prefetch_tensormap(&tmX);
@@ -267,9 +269,9 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         prefetch_tensormap(&tmC);
         prefetch_tensormap(&tmY);
         for (int i = 0; i < Smem::kNumBars; ++i)
-            mbar_init(bars + i, (i >= kEmptyRec && i < kEmptyRec + kCsStages) ? 5u
+            mbar_init(bars + i, (i >= kEmptyRec && i < kEmptyRec + kCsStages) ? (states_only ? 1u : 5u)
                                 : (i >= kFullSt && i < kFullSt + 2)          ? 4u
-                                : (i >= kEmptyCB && i < kEmptyCB + 2)        ? 2u
+                                : (i >= kEmptyCB && i < kEmptyCB + 2)        ? (states_only ? 1u : 2u)
                                                                              : 1u);
         mbar_fence_init();
         *abort_flag = 0;
@@ -319,12 +321,14 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     const int t0 = s.tile * kT;
                     if (elect_one_sync()) {
                         if (pf.valid) tma_prefetch_l2_4d(&tmX, 0, pf.h, pf.tile * kT, pf.b);
-                        mbar_arrive_expect_tx(bars + kFullCB + cb, p.nkh * 2 * 16384);
+                        mbar_arrive_expect_tx(bars + kFullCB + cb,
+                                              p.nkh * (states_only ? 1 : 2) * 16384);
 #pragma unroll
                         for (int q = 0; q < kN / 64; ++q) {
                             if (q >= p.nkh) break;
-                            tma_load_4d(sm + Smem::kC + cb * kTileBytesCB + q * 16384, &tmC, q * 64, g,
-                                        t0, s.b, bars + kFullCB + cb);
+                            if (!states_only)
+                                tma_load_4d(sm + Smem::kC + cb * kTileBytesCB + q * 16384, &tmC, q * 64,
+                                            g, t0, s.b, bars + kFullCB + cb);
                             tma_load_4d(sm + Smem::kB + cb * kTileBytesCB + q * 16384, &tmB, q * 64, g,
                                         t0, s.b, bars + kFullCB + cb);
                         }
@@ -390,9 +394,10 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             const uint64_t dbt = dbt0 + cb * (kTileBytesCB >> 4);
             wait_bar(bars + kFullCB + cb, (k / kCbStages) & 1, abort_flag, p.status);
             // S[sb] held S~ and Ys of tile k-2 until its epilogue read them
-            if (k >= 2) wait_bar(bars + kEmptyY + sb, ((k - 2) >> 1) & 1, abort_flag, p.status);
+            if (k >= 2 && !states_only)
+                wait_bar(bars + kEmptyY + sb, ((k - 2) >> 1) & 1, abort_flag, p.status);
             tc_fence_after_sync();
-            if (elect_one_sync()) {
+            if (!states_only && elect_one_sync()) {
 #pragma unroll
                 for (int q = 0; q < kN / 16; ++q) {
                     if (q >= 4 * p.nkh) break;
@@ -419,7 +424,7 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         if (elect_one_sync()) mma_commit(bars + kDrain);
         __syncwarp();
         mbar_wait(bars + kDrain, 0, kMbarLimit);
-    } else if (warp == kWarpMmaB) {
+    } else if (warp == kWarpMmaB && !states_only) {
         // ----------------------------------------------- stream B: MMA2, MMA3
         constexpr uint32_t id_y2 = idesc_bf16(128, kP, false, true);
         const uint64_t dc0 = sdesc_sw128(smem_addr(sm + Smem::kC), 16, 1024);
@@ -543,9 +548,12 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             }
             fence_async_shared();
             named_bar_sync(kBarPrep, 64);
-            if (t == 0) mbar_arrive(bars + kFullXt);
+            if (t == 0) {
+                mbar_arrive(bars + kFullXt);
+                if (states_only) mbar_arrive(bars + kEmptyX + xs);
+            }
         }
-    } else if (warp >= kWgMask0 && warp < kWgMask0 + 4) {
+    } else if (warp >= kWgMask0 && warp < kWgMask0 + 4 && !states_only) {
         // ------------------------------------------- mask S -> S~ (in place, TMEM)
         // S~ (bf16 pairs) overwrites the first 64 columns of the tile's S: block
         // jb of S~ lands on columns 16 jb .. 16 jb + 15, which hold S values that
@@ -706,8 +714,9 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             const TileRec& r = recs[c];
             wait_bar(bars + kFullRec + c, (k / kCsStages) & 1, abort_flag, p.status);
             const float cs_n = r.cs[n];
-            const float dec = ex2_approx(r.cs[kT - 1]);
-            write_hs(k);
+            const float cs_end = r.cs[kT - 1];
+            const float dec = ex2_approx(cs_end);
+            if (!states_only) write_hs(k);
 
             // h = exp(cs_end) h_prev + s
             wait_bar(bars + kFullStates + sb, (k >> 1) & 1, abort_flag, p.status);
@@ -724,7 +733,7 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             named_bar_sync(kBarOut, 128);
             if (n == 0) mbar_arrive(bars + kEmptyStates + sb);
 
-            if (p.mode == 1) lam += r.cs[kT - 1];
+            if (states_only) lam += cs_end;
             if (last) {
                 if (s.tile == p.ntiles - 1) {
                     if (p.final_state && n_live) {
@@ -751,6 +760,13 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                             st_release_gpu(p.flags + s.chain, static_cast<unsigned int>(s.seg + 1));
                     }
                 }
+            }
+
+            if (states_only) {
+                // no outputs in this pass: the record is free once every output
+                // warp has read it (the named barrier after the state update)
+                if (n == 0) mbar_arrive(bars + kEmptyRec + c);
+                continue;
             }
 
             // epilogue: y_n = Yd_n + exp(cs_n) Ys_n (bf16), staged in shared memory
@@ -787,10 +803,8 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             tc_fence_before_sync();
             named_bar_sync(kBarOut, 128);
             if (n == 0) {
-                if (p.mode != 1) {
-                    tma_store_4d(&tmY, sm + Smem::kYs, 0, s.h, s.tile * kT, s.b);
-                    tma_store_commit();
-                }
+                tma_store_4d(&tmY, sm + Smem::kYs, 0, s.h, s.tile * kT, s.b);
+                tma_store_commit();
                 mbar_arrive(bars + kEmptyY + sb);
                 mbar_arrive(bars + kEmptyRec + c);
             }
