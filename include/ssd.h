@@ -151,13 +151,20 @@ ssd_status ssd_step(const void* x, const float* dt, const float* A, const void* 
                     int P, int G, int N, ssd_dtype dtype, ssd_stream_t stream);
 
 /* Number of kernels one ssd_forward call with these sizes enqueues (0 if the
- * sizes are invalid or there are no tokens): 1 on the tensor-core path; 3 when
- * its chains are cut into eight or more segments (few (batch, head) chains on
- * long sequences: every segment's local state, a scan over the segments, then
- * the outputs); 3 on the SIMT path. Host-side query; it reads the current
- * device's SM count and launches nothing. */
+ * sizes are invalid or there are no tokens): 1 for the tensor-core single
+ * pass; 3 for the segment-parallel form (see ssd_forward_path: every
+ * segment's local state, a scan over the segments, then the outputs); 3 on the
+ * SIMT path. Host-side query; it reads the current device's SM count and
+ * launches nothing. */
 int ssd_forward_kernel_count(int B, int L, int H, int P, int G, int N, int chunk,
                              ssd_dtype dtype);
+
+/* Which path one ssd_forward call with these sizes takes: 0 if the sizes are
+ * invalid or there are no tokens, 1 the SIMT path, 2 the tensor-core single
+ * pass, 3 the tensor-core segment-parallel form (chains cut into eight or more
+ * segments: few (batch, head) chains on long sequences). Host-side query; it
+ * reads the current device's SM count and launches nothing. */
+int ssd_forward_path(int B, int L, int H, int P, int G, int N, int chunk, ssd_dtype dtype);
 
 /* Synchronises `stream`, then reports and clears the device status word:
  * SSD_OK, SSD_ERR_TIMEOUT (a bounded wait gave up in an earlier call), or

@@ -255,6 +255,16 @@ int ssd_forward_kernel_count(int B, int L, int H, int P, int G, int N, int chunk
     return tc_supported(a) ? tc_kernel_count(a) : 3;
 }
 
+int ssd_forward_path(int B, int L, int H, int P, int G, int N, int chunk, ssd_dtype dtype)
+{
+    if (check_dims(B, L, H, P, G, N, chunk, dtype) != SSD_OK) return 0;
+    if ((long long)B * L == 0) return 0;
+    FwdArgs a = make_args(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                          nullptr, B, L, H, P, G, N, chunk, dtype);
+    if (!tc_supported(a)) return 1;
+    return tc_segment_parallel(a) ? 3 : 2;
+}
+
 ssd_status ssd_poll_status(ssd_stream_t stream)
 {
     if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)

@@ -1026,6 +1026,8 @@ size_t tc_workspace_bytes(const FwdArgs& a) { return ws_layout(a, segments(a, sm
 
 int tc_kernel_count(const FwdArgs& a) { return segments(a, sm_count()).parallel ? 3 : 1; }
 
+bool tc_segment_parallel(const FwdArgs& a) { return segments(a, sm_count()).parallel; }
+
 void tc_set_skip_publish(int v) { g_skip_publish = v; }
 
 cudaError_t tc_forward(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)

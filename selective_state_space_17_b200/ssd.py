@@ -43,6 +43,8 @@ lib.ssd_poll_status.argtypes = [_vp]
 lib.ssd_poll_status.restype = _i
 lib.ssd_forward_kernel_count.argtypes = [_i] * 8
 lib.ssd_forward_kernel_count.restype = _i
+lib.ssd_forward_path.argtypes = [_i] * 8
+lib.ssd_forward_path.restype = _i
 lib.ssd_set_fault_injection.argtypes = [_i]
 lib.ssd_set_fault_injection.restype = None
 lib.ssd_set_wait_limit.argtypes = [ctypes.c_uint64]
@@ -157,6 +159,12 @@ def forward(x, dt, A, Bm, Cm, D=None, chunk: int = 256, initial_state=None, y=No
 def kernel_count(B, L, H, P, G, N, chunk, dtype_code) -> int:
     """Kernels one forward call with these sizes launches (host-side query)."""
     return int(lib.ssd_forward_kernel_count(B, L, H, P, G, N, chunk, dtype_code))
+
+
+def forward_path(B, L, H, P, G, N, chunk, dtype_code) -> int:
+    """Path of one forward call with these sizes (host-side query): 0 invalid or
+    empty, 1 SIMT, 2 tensor-core single pass, 3 tensor-core segment-parallel."""
+    return int(lib.ssd_forward_path(B, L, H, P, G, N, chunk, dtype_code))
 
 
 def forward_host_buffer_size(B, L, H, P, G, N, chunk, dtype_code) -> int:

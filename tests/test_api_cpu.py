@@ -36,6 +36,17 @@ def test_library_exports_every_declared_entry_point(lib):
         assert hasattr(lib, n), f"{n} declared in include/ but not exported"
 
 
+def test_forward_path_query(lib):
+    # bf16 with P = 64 and N <= 128 takes the tensor-core path; few chains on a
+    # long sequence run segment-parallel; fp32 takes the SIMT path
+    assert lib.ssd_forward_path(4, 4096, 80, 64, 1, 128, 256, 1) == 2
+    assert lib.ssd_forward_path(1, 4096, 4, 64, 1, 128, 256, 1) == 3
+    assert lib.ssd_forward_path(1, 64, 2, 8, 1, 8, 16, 0) == 1
+    assert lib.ssd_forward_path(1, 512, 2, 64, 1, 256, 128, 1) == 1   # N = 256: SIMT
+    assert lib.ssd_forward_path(1, 64, 3, 8, 2, 8, 16, 0) == 0        # H % G != 0
+    assert lib.ssd_forward_path(0, 64, 2, 8, 1, 8, 16, 0) == 0        # no tokens
+
+
 def test_status_strings(lib):
     for code in range(7):
         s = lib.ssd_status_string(code).decode()

@@ -23,8 +23,9 @@ def ssd():
 
 def test_bench_workload_takes_the_tensor_core_path(ssd):
     w = gen.LAYER_2P7B
+    assert ssd.forward_path(w.B, w.L, w.H, w.P, w.G, w.N, w.chunk, ssd.SSD_BF16) == 2
     assert ssd.kernel_count(w.B, w.L, w.H, w.P, w.G, w.N, w.chunk, ssd.SSD_BF16) == 1
-    assert ssd.kernel_count(1, 64, 2, 8, 1, 8, 16, ssd.SSD_F32) == 3
+    assert ssd.forward_path(1, 64, 2, 8, 1, 8, 16, ssd.SSD_F32) == 1
 
 
 def test_lookback_timeout_is_reported_and_context_survives(ssd, oracle):

@@ -88,7 +88,7 @@ def test_tensor_core_state_dims(ssd, oracle, N, chunk):
     inp = gen.make_inputs(2, 300, 4, 64, 2, N, "bf16", seed=9)
     rng = np.random.default_rng(1)
     init = rng.standard_normal((2, 4, 64, N)).astype(np.float32)
-    assert ssd.kernel_count(2, 300, 4, 64, 2, N, chunk, 1) == 1
+    assert ssd.forward_path(2, 300, 4, 64, 2, N, chunk, 1) == 2
     _full_check(ssd, oracle, inp, chunk, init=init)
 
 
@@ -99,7 +99,7 @@ def test_tensor_core_state_dims(ssd, oracle, N, chunk):
 def test_segment_parallel_form(ssd, oracle, shape, chunk, with_init):
     """Few chains with many tiles: each segment's local state, a scan over the
     segments, then the outputs (three launches instead of a serial look-back)."""
-    assert ssd.kernel_count(*shape, chunk, 1) == 3
+    assert ssd.forward_path(*shape, chunk, 1) == 3
     inp = gen.make_inputs(*shape, "bf16", seed=10)
     init = None
     if with_init:
