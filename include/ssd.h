@@ -92,10 +92,14 @@ size_t ssd_workspace_size(int B, int L, int H, int P, int G, int N, int chunk, s
  *   initial_state or 0), H >= 1, G >= 1, H % G == 0, P in [1, 256],
  *   N in [1, 256]. All pointers 16-byte aligned.
  *   The tensor-core path is taken for bf16 with P == 64, N a multiple of 8
- *   with 8 <= N <= 128, and chunk in {64, 128, 256}; other valid sizes run
+ *   with 8 <= N <= 256, and chunk in {64, 128, 256}; other valid sizes run
  *   the SIMT path. The tensor-core path evaluates the chunked form on
  *   128-token tiles whatever `chunk` is (the result does not depend on the
- *   chunk length beyond rounding).
+ *   chunk length beyond rounding). With N > 128 it runs two passes over the
+ *   state columns (n < 128, then the rest; each state column evolves on its
+ *   own and y is a sum over columns): the first stores y with the D term,
+ *   the second adds its share into y in L2 (a bf16 add, so y is rounded
+ *   twice), and each writes its columns of final_state.
  */
 ssd_status ssd_forward(const void* x, const float* dt, const float* A, const void* Bm,
                        const void* Cm, const float* D, const float* initial_state, void* y,
@@ -111,7 +115,7 @@ ssd_status ssd_forward(const void* x, const float* dt, const float* A, const voi
  * ring, 256 + 4*B*H rounded to 256 + 2*B*H*64*128*4 bytes) lives in a fixed
  * 24 MiB device array inside the library, which every GPU that loads the
  * library holds until the process exits. Only the tensor-core sizes are
- * handled (bf16, P == 64, N a multiple of 8 up to 128, chunk 64, 128 or 256,
+ * handled (bf16, P == 64, N a multiple of 8 up to 256, chunk 64, 128 or 256,
  * B*L > 0); other sizes return SSD_ERR_UNSUPPORTED, and sizes whose scratch
  * exceeds the array (B*H > 383) return SSD_ERR_WORKSPACE before anything is
  * enqueued. The call allocates nothing. The first call on each device looks
@@ -153,8 +157,9 @@ ssd_status ssd_step(const void* x, const float* dt, const float* A, const void* 
 /* Number of kernels one ssd_forward call with these sizes enqueues (0 if the
  * sizes are invalid or there are no tokens): 1 for the tensor-core single
  * pass; 3 for the segment-parallel form (see ssd_forward_path: every
- * segment's local state, a scan over the segments, then the outputs); 3 on the
- * SIMT path. Host-side query; it reads the current device's SM count and
+ * segment's local state, a scan over the segments, then the outputs); twice
+ * that on the tensor-core path when N > 128 (one pass per 128 state
+ * columns); 3 on the SIMT path. Host-side query; it reads the current device's SM count and
  * launches nothing. */
 int ssd_forward_kernel_count(int B, int L, int H, int P, int G, int N, int chunk,
                              ssd_dtype dtype);

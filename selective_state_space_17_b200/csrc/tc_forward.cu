@@ -123,8 +123,15 @@ struct TcParams {
     unsigned int* status;
     unsigned long long wait_limit;
     int B, L, H, G;
-    int N;        // state dim (<= kN)
-    int nkh;      // 64-wide halves of the state dim that hold data (1 or 2)
+    // A state dim above kN runs as two passes over the state columns
+    // [n_off, n_off + N): the output is linear in the state columns (y sums
+    // C_i,n h_n and the masked C_i,n B_j,n over n), so the second pass adds its
+    // share into y (TMA reduce-add) and leaves out the D x term.
+    int N;        // state columns of this pass (<= kN)
+    int n_off;    // first state column of this pass
+    int ldn;      // state dim of Bm, Cm, initial and final state
+    int accumulate;  // 1: add into y instead of storing it
+    int nkh;      // 64-wide halves of the pass's state columns that hold data (1 or 2)
     int ntiles;   // tiles per chain
     int chains;   // B * H
     int seg_len;  // tiles per segment
@@ -327,9 +334,9 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                         for (int q = 0; q < kN / 64; ++q) {
                             if (q >= p.nkh) break;
                             if (!states_only)
-                                tma_load_4d(sm + Smem::kC + cb * kTileBytesCB + q * 16384, &tmC, q * 64,
+                                tma_load_4d(sm + Smem::kC + cb * kTileBytesCB + q * 16384, &tmC, p.n_off + q * 64,
                                             g, t0, s.b, bars + kFullCB + cb);
-                            tma_load_4d(sm + Smem::kB + cb * kTileBytesCB + q * 16384, &tmB, q * 64, g,
+                            tma_load_4d(sm + Smem::kB + cb * kTileBytesCB + q * 16384, &tmB, p.n_off + q * 64, g,
                                         t0, s.b, bars + kFullCB + cb);
                         }
                     }
@@ -635,8 +642,8 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         const int wq = warp - kWgOut0;
         const int n = wq * 32 + lane;  // state row / tile row / TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-        const size_t PN = static_cast<size_t>(kP) * p.N;
-        const bool n_live = n < p.N;  // rows past N are zero padding
+        const size_t PN = static_cast<size_t>(kP) * p.ldn;
+        const bool n_live = n < p.N;  // rows past the pass's columns are zero padding
         float h[kP];
         float lam = 0.f;  // log2 decay of the segment so far (mode 1)
         // the bf16 h_prev operand of MMA3 for tile kk (row n of [N][P],
@@ -672,9 +679,9 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
 #pragma unroll
                     for (int q = 0; q < kP; ++q) h[q] = 0.f;
                 } else if (s.seg == 0) {
-                    const float* src = p.init + static_cast<size_t>(s.chain) * PN;
+                    const float* src = p.init + static_cast<size_t>(s.chain) * PN + p.n_off + n;
 #pragma unroll
-                    for (int q = 0; q < kP; ++q) h[q] = n_live ? src[static_cast<size_t>(q) * p.N + n] : 0.f;
+                    for (int q = 0; q < kP; ++q) h[q] = n_live ? src[static_cast<size_t>(q) * p.ldn] : 0.f;
                 } else {
                     if (p.mode == 0) {
                         if (n == 0 && !*abort_flag) {
@@ -737,9 +744,9 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             if (last) {
                 if (s.tile == p.ntiles - 1) {
                     if (p.final_state && n_live) {
-                        float* dst = p.final_state + static_cast<size_t>(s.chain) * PN;
+                        float* dst = p.final_state + static_cast<size_t>(s.chain) * PN + p.n_off + n;
 #pragma unroll
-                        for (int q = 0; q < kP; ++q) dst[static_cast<size_t>(q) * p.N + n] = h[q];
+                        for (int q = 0; q < kP; ++q) dst[static_cast<size_t>(q) * p.ldn] = h[q];
                     }
                 } else if (p.mode != 2) {
                     // mode 0 publishes the segment's end state to the ring; mode 1
@@ -803,7 +810,10 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             tc_fence_before_sync();
             named_bar_sync(kBarOut, 128);
             if (n == 0) {
-                tma_store_4d(&tmY, sm + Smem::kYs, 0, s.h, s.tile * kT, s.b);
+                if (p.accumulate)
+                    tma_reduce_add_4d(&tmY, sm + Smem::kYs, 0, s.h, s.tile * kT, s.b);
+                else
+                    tma_store_4d(&tmY, sm + Smem::kYs, 0, s.h, s.tile * kT, s.b);
                 tma_store_commit();
                 mbar_arrive(bars + kEmptyY + sb);
                 mbar_arrive(bars + kEmptyRec + c);
@@ -934,18 +944,19 @@ int g_skip_publish = 0;
 // states and decays: h_in(0) = initial state, h_in(s + 1) = 2^decay(s) h_in(s)
 // + local(s) (the composition of affine maps of "Selective SSM guide", eq. (3),
 // applied segment by segment). One thread per state element of a chain
-// (blockIdx.y = chain); states are [kN][kP] with rows past N zero.
+// (blockIdx.y = chain); states are [kN][kP] with rows past N zero, and the
+// initial state's columns [n_off, n_off + N) of its ldn feed this pass.
 constexpr int kScanThreads = 256;
 static_assert(kN * kP % kScanThreads == 0, "scan grid covers the state exactly");
 
 __global__ void __launch_bounds__(kScanThreads)
 segment_scan_kernel(const float* init, const float* seg_state, const float* seg_decay,
-                    float* seg_hin, int P, int N, int nseg)
+                    float* seg_hin, int P, int N, int n_off, int ldn, int nseg)
 {
     const size_t chain = blockIdx.y;
     const int e = blockIdx.x * kScanThreads + threadIdx.x;  // < kN * kP by the grid
     const int n = e / kP, q = e - n * kP;
-    float v = init && n < N ? init[(chain * P + q) * N + n] : 0.f;
+    float v = init && n < N ? init[(chain * P + q) * ldn + n_off + n] : 0.f;
     const size_t u0 = chain * nseg;
 #pragma unroll 8
     for (int sg = 0; sg < nseg; ++sg) {
@@ -984,8 +995,7 @@ cudaError_t launch(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)
     p.L = a.L;
     p.H = a.H;
     p.G = a.G;
-    p.N = a.N;
-    p.nkh = a.N <= 64 ? 1 : 2;
+    p.ldn = a.N;
     p.ntiles = g.ntiles;
     p.chains = g.chains;
     p.seg_len = g.seg_len;
@@ -1002,21 +1012,34 @@ cudaError_t launch(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)
         tc_forward_kernel<<<grid, kThreads, smem, ctx.stream>>>(tmX, tmB, tmC, tmY, p);
         return cudaGetLastError();
     };
-    if (!g.parallel) return run(0, g.chains * g.nseg);
-    // segment-parallel: local states of every segment but each chain's last
-    // (segment-major numbering puts those first), the scan, then the outputs
-    if ((e = run(1, g.chains * (g.nseg - 1))) != cudaSuccess) return e;
-    segment_scan_kernel<<<dim3(kN * kP / kScanThreads, g.chains), kScanThreads, 0, ctx.stream>>>(
-        a.init, p.seg_state, p.seg_decay, reinterpret_cast<float*>(ws + w.seg_hin), kP, a.N, g.nseg);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    return run(2, g.chains * g.nseg);
+    // one pass per kN state columns; every pass after the first adds into y
+    for (int n_off = 0; n_off < a.N; n_off += kN) {
+        p.n_off = n_off;
+        p.N = a.N - n_off < kN ? a.N - n_off : kN;
+        p.nkh = p.N <= 64 ? 1 : 2;
+        p.accumulate = n_off > 0;
+        p.D = n_off > 0 ? nullptr : a.D;
+        if (!g.parallel) {
+            if ((e = run(0, g.chains * g.nseg)) != cudaSuccess) return e;
+            continue;
+        }
+        // segment-parallel: local states of every segment but each chain's last
+        // (segment-major numbering puts those first), the scan, then the outputs
+        if ((e = run(1, g.chains * (g.nseg - 1))) != cudaSuccess) return e;
+        segment_scan_kernel<<<dim3(kN * kP / kScanThreads, g.chains), kScanThreads, 0, ctx.stream>>>(
+            a.init, p.seg_state, p.seg_decay, reinterpret_cast<float*>(ws + w.seg_hin), kP, p.N,
+            n_off, a.N, g.nseg);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if ((e = run(2, g.chains * g.nseg)) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace
 
 bool tc_supported(const FwdArgs& a)
 {
-    return a.bf16 && a.P == kP && a.N % 8 == 0 && a.N >= 8 && a.N <= kN &&
+    return a.bf16 && a.P == kP && a.N % 8 == 0 && a.N >= 8 && a.N <= 2 * kN &&
            (a.chunk == 64 || a.chunk == 128 || a.chunk == 256) &&
            static_cast<long long>(a.B) * a.L > 0 &&
            static_cast<long long>((a.L + kT - 1) / kT) * a.B * a.H < (1ll << 31);
@@ -1024,7 +1047,12 @@ bool tc_supported(const FwdArgs& a)
 
 size_t tc_workspace_bytes(const FwdArgs& a) { return ws_layout(a, segments(a, sm_count())).total; }
 
-int tc_kernel_count(const FwdArgs& a) { return segments(a, sm_count()).parallel ? 3 : 1; }
+int tc_passes(const FwdArgs& a) { return (a.N + kN - 1) / kN; }
+
+int tc_kernel_count(const FwdArgs& a)
+{
+    return tc_passes(a) * (segments(a, sm_count()).parallel ? 3 : 1);
+}
 
 bool tc_segment_parallel(const FwdArgs& a) { return segments(a, sm_count()).parallel; }
 

@@ -37,14 +37,26 @@ def test_library_exports_every_declared_entry_point(lib):
 
 
 def test_forward_path_query(lib):
-    # bf16 with P = 64 and N <= 128 takes the tensor-core path; few chains on a
-    # long sequence run segment-parallel; fp32 takes the SIMT path
+    # bf16 with P = 64 and N a multiple of 8 up to 256 takes the tensor-core
+    # path; few chains on a long sequence run segment-parallel; fp32 and other
+    # sizes take the SIMT path
     assert lib.ssd_forward_path(4, 4096, 80, 64, 1, 128, 256, 1) == 2
     assert lib.ssd_forward_path(1, 4096, 4, 64, 1, 128, 256, 1) == 3
     assert lib.ssd_forward_path(1, 64, 2, 8, 1, 8, 16, 0) == 1
-    assert lib.ssd_forward_path(1, 512, 2, 64, 1, 256, 128, 1) == 1   # N = 256: SIMT
+    assert lib.ssd_forward_path(1, 512, 2, 64, 1, 256, 128, 1) == 2   # N = 256: two passes
+    assert lib.ssd_forward_path(1, 512, 2, 64, 1, 252, 128, 1) == 1   # N % 8 != 0: SIMT
+    assert lib.ssd_forward_path(1, 512, 2, 32, 1, 128, 128, 1) == 1   # P != 64: SIMT
     assert lib.ssd_forward_path(1, 64, 3, 8, 2, 8, 16, 0) == 0        # H % G != 0
     assert lib.ssd_forward_path(0, 64, 2, 8, 1, 8, 16, 0) == 0        # no tokens
+
+
+def test_kernel_count_query(lib):
+    # one launch per 128 state columns on the tensor-core single pass (no SM
+    # count is readable here, so the query assumes 148)
+    assert lib.ssd_forward_kernel_count(1, 512, 2, 64, 1, 128, 128, 1) == 1
+    assert lib.ssd_forward_kernel_count(1, 512, 2, 64, 1, 256, 128, 1) == 2
+    assert lib.ssd_forward_kernel_count(1, 4096, 4, 64, 1, 200, 256, 1) == 6
+    assert lib.ssd_forward_kernel_count(1, 64, 2, 8, 1, 8, 16, 0) == 3
 
 
 def test_status_strings(lib):

@@ -81,20 +81,24 @@ def test_special_cases(ssd, oracle, kind, dtype):
     _full_check(ssd, oracle, inp, 128 if dtype == "bf16" else 64)
 
 
-@pytest.mark.parametrize("N,chunk", [(8, 64), (48, 128), (64, 256), (96, 64), (120, 128)])
+@pytest.mark.parametrize("N,chunk", [(8, 64), (48, 128), (64, 256), (96, 64), (120, 128),
+                                     (136, 64), (200, 128), (256, 256)])
 def test_tensor_core_state_dims(ssd, oracle, N, chunk):
     """State dims below 128 run on the tensor-core path with the state rows
-    zero-padded to 128 (a ragged tail, an initial state and two groups too)."""
+    zero-padded to 128; above 128 as two passes over the state columns, the
+    second adding into y (a ragged tail, an initial state and two groups too)."""
     inp = gen.make_inputs(2, 300, 4, 64, 2, N, "bf16", seed=9)
     rng = np.random.default_rng(1)
     init = rng.standard_normal((2, 4, 64, N)).astype(np.float32)
     assert ssd.forward_path(2, 300, 4, 64, 2, N, chunk, 1) == 2
+    assert ssd.kernel_count(2, 300, 4, 64, 2, N, chunk, 1) == (2 if N > 128 else 1)
     _full_check(ssd, oracle, inp, chunk, init=init)
 
 
 @pytest.mark.parametrize("shape,chunk,with_init", [
     ((1, 4096, 4, 64, 1, 128), 256, False),   # 4 chains of 32 tiles: one tile per segment
     ((2, 3000, 2, 64, 1, 64), 128, True),     # ragged tail, N = 64, initial state
+    ((1, 3000, 2, 64, 2, 192), 256, True),    # N = 192: two passes of three launches
 ])
 def test_segment_parallel_form(ssd, oracle, shape, chunk, with_init):
     """Few chains with many tiles: each segment's local state, a scan over the

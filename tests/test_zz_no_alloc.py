@@ -44,7 +44,8 @@ def _noalloc(ssd, t, y, fs, shape, chunk, stream):
 def test_noalloc_matches_workspace_entry_point_on_two_calls(ssd):
     stream = torch.cuda.current_stream()
     cases = [((2, 1000, 8, 64, 1, 128), 256, 31),  # ragged last tile
-             ((1, 640, 6, 64, 2, 128), 128, 32)]
+             ((1, 640, 6, 64, 2, 128), 128, 32),
+             ((1, 640, 4, 64, 2, 256), 128, 35)]   # two passes over the state columns
     for shape, chunk, seed in cases:
         inp = gen.make_inputs(*shape, "bf16", seed=seed)
         t = to_device(inp)
@@ -69,11 +70,11 @@ def test_noalloc_refuses_what_it_cannot_run(ssd):
     y = torch.empty_like(t["x"])
     fs = torch.empty((8, 64, 64, 128), dtype=torch.float32, device="cuda")
     assert _noalloc(ssd, t, y, fs, big, 128, stream) == 6  # SSD_ERR_WORKSPACE
-    # N = 256 is not a tensor-core size (the tiles hold N <= 128)
-    small = (1, 256, 2, 64, 1, 256)
+    # P = 32 is not a tensor-core size (the tiles hold P = 64)
+    small = (1, 256, 2, 32, 1, 128)
     t = to_device(gen.make_inputs(*small, "bf16", seed=34))
     y = torch.empty_like(t["x"])
-    fs = torch.empty((1, 2, 64, 256), dtype=torch.float32, device="cuda")
+    fs = torch.empty((1, 2, 32, 128), dtype=torch.float32, device="cuda")
     assert _noalloc(ssd, t, y, fs, small, 128, stream) == 2  # SSD_ERR_UNSUPPORTED
     torch.cuda.synchronize()
     assert np.isfinite(to_host_f64(t["x"][:1, :1])).all()
