@@ -166,8 +166,9 @@ int ssd_forward_kernel_count(int B, int L, int H, int P, int G, int N, int chunk
 
 /* Which path one ssd_forward call with these sizes takes: 0 if the sizes are
  * invalid or there are no tokens, 1 the SIMT path, 2 the tensor-core single
- * pass, 3 the tensor-core segment-parallel form (chains cut into eight or more
- * segments: few (batch, head) chains on long sequences). Host-side query; it
+ * pass, 3 the tensor-core segment-parallel form (fewer (batch, head) chains
+ * than half the SMs, each cut into eight or more segments: few chains on long
+ * sequences). Host-side query; it
  * reads the current device's SM count and launches nothing. */
 int ssd_forward_path(int B, int L, int H, int P, int G, int N, int chunk, ssd_dtype dtype);
 
