@@ -91,7 +91,9 @@ size_t ssd_workspace_size(int B, int L, int H, int P, int G, int N, int chunk, s
  *   Sizes: B, L >= 0 (B*L == 0 is a no-op apart from final_state =
  *   initial_state or 0), H >= 1, G >= 1, H % G == 0, P in [1, 256],
  *   N in [1, 256]. All pointers 16-byte aligned.
- *   The tensor-core path is taken for bf16 with P == 64, N a multiple of 8
+ *   The tensor-core path is taken for bf16 with P a multiple of 64 (a head of
+ *   P = 64m channels runs as m heads of 64 channels sharing dt, A and D: the
+ *   rows of the P x N state evolve independently), N a multiple of 8
  *   with 8 <= N <= 256, and chunk in {64, 128, 256}; other valid sizes run
  *   the SIMT path. The tensor-core path evaluates the chunked form on
  *   128-token tiles whatever `chunk` is (the result does not depend on the
@@ -112,12 +114,14 @@ ssd_status ssd_forward(const void* x, const float* dt, const float* A, const voi
  * device memory. The pages describe no such entry point; it is a convenience
  * of this library. It takes the same arguments as ssd_forward without the
  * workspace: its scratch (look-back control words and the per-head state
- * ring, 256 + 4*B*H rounded to 256 + 2*B*H*64*128*4 bytes) lives in a fixed
+ * ring, with M = B*H*P/64: 256 + 4*M rounded to 256, + 2*M*64*128*4 bytes) lives in a fixed
  * 24 MiB device array inside the library, which every GPU that loads the
  * library holds until the process exits. Only the tensor-core sizes are
- * handled (bf16, P == 64, N a multiple of 8 up to 256, chunk 64, 128 or 256,
+ * handled (bf16, P a multiple of 64, N a multiple of 8 up to 256, chunk 64, 128 or 256,
  * B*L > 0); other sizes return SSD_ERR_UNSUPPORTED, and sizes whose scratch
- * exceeds the array (B*H > 383) return SSD_ERR_WORKSPACE before anything is
+ * exceeds the array (M > 383; or, in the segment-parallel form, the two
+ * per-segment states, 2*M*nseg*64*128*4 more bytes, see ssd_workspace_size)
+ * return SSD_ERR_WORKSPACE before anything is
  * enqueued. The call allocates nothing. The first call on each device looks
  * up the array's device address (make it before any stream capture). All
  * calls on a device share the array: calls that may overlap on the GPU race

@@ -122,7 +122,14 @@ struct TcParams {
     const float* seg_hin; // [chain][seg][kN][kP]
     unsigned int* status;
     unsigned long long wait_limit;
-    int B, L, H, G;
+    int B, L, G;
+    // A head with P = sub * kP channels runs as `sub` heads of kP channels
+    // (each row of the P x N state evolves on its own, and x, y [B][L][H][P]
+    // and the states [B][H][P][N] read as [B][L][H sub][kP] and
+    // [B][H sub][kP][N]); those share the head's dt, A and D.
+    int H;        // heads of kP channels (H_model * sub)
+    int Hr;       // heads of the model: dt [B][L][Hr], A and D [Hr]
+    int sub;      // kP-channel heads per model head
     // A state dim above kN runs as two passes over the state columns
     // [n_off, n_off + N): the output is linear in the state columns (y sums
     // C_i,n h_n and the masked C_i,n B_j,n over n), so the second pass adds its
@@ -485,11 +492,12 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         float A_next = 0.f, D_next = 0.f;
         auto fetch = [&](const Seq& q) {
             const int rows = min(kT, p.L - q.tile * kT);
-            const size_t base = (static_cast<size_t>(q.b) * p.L + q.tile * kT) * p.H + q.h;
-            dt_next.x = 2 * t < rows ? p.dt[base + static_cast<size_t>(2 * t) * p.H] : 0.f;
-            dt_next.y = 2 * t + 1 < rows ? p.dt[base + static_cast<size_t>(2 * t + 1) * p.H] : 0.f;
-            A_next = p.A[q.h];
-            D_next = p.D ? p.D[q.h] : 0.f;
+            const int hr = p.sub == 1 ? q.h : q.h / p.sub;  // the model head
+            const size_t base = (static_cast<size_t>(q.b) * p.L + q.tile * kT) * p.Hr + hr;
+            dt_next.x = 2 * t < rows ? p.dt[base + static_cast<size_t>(2 * t) * p.Hr] : 0.f;
+            dt_next.y = 2 * t + 1 < rows ? p.dt[base + static_cast<size_t>(2 * t + 1) * p.Hr] : 0.f;
+            A_next = p.A[hr];
+            D_next = p.D ? p.D[hr] : 0.f;
         };
         if (s.valid) fetch(s);
         for (int k = 0; s.valid; ++k) {
@@ -873,6 +881,9 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint
     return r == CUDA_SUCCESS;
 }
 
+// Heads of kP channels: a model head of P = sub * kP channels is sub of them.
+int tile_heads(const FwdArgs& a) { return a.H * (a.P / kP); }
+
 // Segments per chain: enough items for about eight per CTA, at least one tile each.
 void choose_segments(int ntiles, int chains, int ctas, int* seg_len, int* nseg)
 {
@@ -912,7 +923,7 @@ Segments segments(const FwdArgs& a, int ctas)
 {
     Segments g;
     g.ntiles = (a.L + kT - 1) / kT;
-    g.chains = a.B * a.H;
+    g.chains = a.B * tile_heads(a);
     choose_segments(g.ntiles, g.chains, ctas, &g.seg_len, &g.nseg);
     g.parallel = g.nseg >= kParallelSegments && 2 * g.chains < ctas;
     return g;
@@ -925,7 +936,7 @@ struct WsLayout {
 WsLayout ws_layout(const FwdArgs& a, const Segments& g)
 {
     WsLayout w;
-    const size_t chains = static_cast<size_t>(a.B) * a.H;
+    const size_t chains = static_cast<size_t>(a.B) * tile_heads(a);
     const size_t slot = static_cast<size_t>(kP) * kN * sizeof(float);
     w.ctrl = 0;
     w.flags = 256;
@@ -973,8 +984,9 @@ segment_scan_kernel(const float* init, const float* seg_state, const float* seg_
 cudaError_t launch(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)
 {
     CUtensorMap tmX, tmB, tmC, tmY;
-    if (!make_map(&tmX, a.x, kP, a.H, a.L, a.B) || !make_map(&tmB, a.Bm, a.N, a.G, a.L, a.B) ||
-        !make_map(&tmC, a.Cm, a.N, a.G, a.L, a.B) || !make_map(&tmY, a.y, kP, a.H, a.L, a.B))
+    const int Ht = tile_heads(a);
+    if (!make_map(&tmX, a.x, kP, Ht, a.L, a.B) || !make_map(&tmB, a.Bm, a.N, a.G, a.L, a.B) ||
+        !make_map(&tmC, a.Cm, a.N, a.G, a.L, a.B) || !make_map(&tmY, a.y, kP, Ht, a.L, a.B))
         return cudaErrorInvalidValue;
     const int ctas_max = ctx.num_sms > 0 ? ctx.num_sms : 1;
     const Segments g = segments(a, ctas_max);
@@ -997,7 +1009,9 @@ cudaError_t launch(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)
     p.wait_limit = ctx.wait_limit;
     p.B = a.B;
     p.L = a.L;
-    p.H = a.H;
+    p.H = Ht;
+    p.Hr = a.H;
+    p.sub = a.P / kP;
     p.G = a.G;
     p.ldn = a.N;
     p.ntiles = g.ntiles;
@@ -1043,10 +1057,10 @@ cudaError_t launch(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)
 
 bool tc_supported(const FwdArgs& a)
 {
-    return a.bf16 && a.P == kP && a.N % 8 == 0 && a.N >= 8 && a.N <= 2 * kN &&
+    return a.bf16 && a.P % kP == 0 && a.P >= kP && a.N % 8 == 0 && a.N >= 8 && a.N <= 2 * kN &&
            (a.chunk == 64 || a.chunk == 128 || a.chunk == 256) &&
            static_cast<long long>(a.B) * a.L > 0 &&
-           static_cast<long long>((a.L + kT - 1) / kT) * a.B * a.H < (1ll << 31);
+           static_cast<long long>((a.L + kT - 1) / kT) * a.B * a.H * (a.P / kP) < (1ll << 31);
 }
 
 size_t tc_workspace_bytes(const FwdArgs& a) { return ws_layout(a, segments(a, sm_count())).total; }

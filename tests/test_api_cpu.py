@@ -45,7 +45,9 @@ def test_forward_path_query(lib):
     assert lib.ssd_forward_path(1, 64, 2, 8, 1, 8, 16, 0) == 1
     assert lib.ssd_forward_path(1, 512, 2, 64, 1, 256, 128, 1) == 2   # N = 256: two passes
     assert lib.ssd_forward_path(1, 512, 2, 64, 1, 252, 128, 1) == 1   # N % 8 != 0: SIMT
-    assert lib.ssd_forward_path(1, 512, 2, 32, 1, 128, 128, 1) == 1   # P != 64: SIMT
+    assert lib.ssd_forward_path(1, 512, 2, 32, 1, 128, 128, 1) == 1   # P = 32: SIMT
+    assert lib.ssd_forward_path(1, 512, 2, 128, 1, 128, 128, 1) == 2  # P = 128: two 64-wide heads
+    assert lib.ssd_forward_path(1, 512, 2, 96, 1, 128, 128, 1) == 1   # P = 96: SIMT
     assert lib.ssd_forward_path(1, 64, 3, 8, 2, 8, 16, 0) == 0        # H % G != 0
     assert lib.ssd_forward_path(0, 64, 2, 8, 1, 8, 16, 0) == 0        # no tokens
 

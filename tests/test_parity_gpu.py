@@ -120,6 +120,22 @@ def test_tensor_core_mixed_decay(ssd, oracle, shape):
     _full_check(ssd, oracle, inp, 128)
 
 
+@pytest.mark.parametrize("shape,chunk", [
+    ((2, 300, 4, 128, 2, 128), 128),   # P = 128: two 64-channel heads per head
+    ((1, 200, 3, 192, 3, 200), 64),    # P = 192 with N = 200 (two passes)
+    ((1, 3000, 2, 128, 1, 64), 256),   # P = 128, segment-parallel
+])
+def test_tensor_core_wide_heads(ssd, oracle, shape, chunk):
+    """Heads of P = 64m channels run on the tensor-core path as m heads of 64
+    channels that share dt, A and D (with an initial state, so its layout is
+    checked too)."""
+    B, L, H, P, G, N = shape
+    assert ssd.forward_path(*shape, chunk, 1) in (2, 3)
+    inp = gen.make_inputs(*shape, "bf16", seed=12)
+    init = np.random.default_rng(3).standard_normal((B, H, P, N)).astype(np.float32)
+    _full_check(ssd, oracle, inp, chunk, init=init)
+
+
 def test_initial_state_and_no_skip_term(ssd, oracle):
     inp = gen.make_inputs(2, 384, 4, 64, 1, 128, "bf16", seed=6)
     rng = np.random.default_rng(0)
