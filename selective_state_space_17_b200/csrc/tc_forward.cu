@@ -90,7 +90,7 @@ constexpr int kBarOut = 2;
 constexpr int kCbStages = 2;
 constexpr int kXStages = 2;
 constexpr int kCsStages = 4;
-constexpr int kPrefetchAhead = 4;
+constexpr int kPrefetchAhead = 2;
 
 // TMEM columns (fp32, 128 lanes)
 constexpr uint32_t kColS = 0;     // 2 x 128: S, then S~ (bf16, cols 0-63) and Ys (cols 64-127)
@@ -884,10 +884,11 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint
 // Heads of kP channels: a model head of P = sub * kP channels is sub of them.
 int tile_heads(const FwdArgs& a) { return a.H * (a.P / kP); }
 
-// Segments per chain: enough items for about eight per CTA, at least one tile each.
-void choose_segments(int ntiles, int chains, int ctas, int* seg_len, int* nseg)
+// Segments per chain: enough items for about `per_cta` per CTA, at least one
+// tile each.
+void choose_segments(int ntiles, int chains, int ctas, int per_cta, int* seg_len, int* nseg)
 {
-    long long want = (8ll * ctas + chains - 1) / chains;
+    long long want = (static_cast<long long>(per_cta) * ctas + chains - 1) / chains;
     if (want < 1) want = 1;
     if (want > ntiles) want = ntiles;
     *seg_len = static_cast<int>((ntiles + want - 1) / want);
@@ -902,6 +903,12 @@ void choose_segments(int ntiles, int chains, int ctas, int* seg_len, int* nseg)
 // (Measured: 32 chains of 512 tiles 1.60 ms single pass, 0.70 ms parallel;
 // 128 chains of 64 tiles 0.26 ms single pass, 0.43 ms parallel.)
 constexpr int kParallelSegments = 8;
+// Items per CTA: the single pass takes about four (each segment boundary
+// costs a state hand-off, and four rounds still balance: 4.3 items per CTA
+// at 320 chains ran 4% faster than 8.6, and 12 or 16 ran slower); the
+// segment-parallel form, whose segments do not wait on each other, about eight.
+constexpr int kItemsPerCtaSingle = 4;
+constexpr int kItemsPerCtaParallel = 8;
 
 int sm_count()
 {
@@ -924,8 +931,9 @@ Segments segments(const FwdArgs& a, int ctas)
     Segments g;
     g.ntiles = (a.L + kT - 1) / kT;
     g.chains = a.B * tile_heads(a);
-    choose_segments(g.ntiles, g.chains, ctas, &g.seg_len, &g.nseg);
+    choose_segments(g.ntiles, g.chains, ctas, kItemsPerCtaSingle, &g.seg_len, &g.nseg);
     g.parallel = g.nseg >= kParallelSegments && 2 * g.chains < ctas;
+    if (g.parallel) choose_segments(g.ntiles, g.chains, ctas, kItemsPerCtaParallel, &g.seg_len, &g.nseg);
     return g;
 }
 
