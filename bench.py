@@ -89,18 +89,49 @@ def combine_ranks(local_ms: float, tokens_per_rank: int, world: int, dist=None, 
     return ms, tokens_per_rank * world / (ms / 1e3) / 1e6
 
 
+def code_digest(paths) -> str:
+    """sha256 over the given C/C++/CUDA sources with comments removed and
+    whitespace collapsed: it changes with the code and not with its comments."""
+    import hashlib
+    h = hashlib.sha256()
+    for path in paths:
+        with open(os.path.join(ROOT, path), encoding="utf-8") as f:
+            text = f.read()
+        out, i, n = [], 0, len(text)
+        while i < n:
+            c = text[i]
+            if text.startswith("//", i):
+                j = text.find("\n", i)
+                i = n if j < 0 else j
+            elif text.startswith("/*", i):
+                j = text.find("*/", i + 2)
+                i = n if j < 0 else j + 2
+                out.append(" ")
+            elif c in "\"'":
+                j = i + 1
+                while j < n and text[j] != c:
+                    j += 2 if text[j] == "\\" else 1
+                out.append(text[i:j + 1])
+                i = j + 1
+            else:
+                out.append(c)
+                i += 1
+        h.update(" ".join("".join(out).split()).encode())
+        h.update(b"\0")
+    return h.hexdigest()
+
+
 def recorded_traffic(workload: str):
     """DRAM bytes (read + write) of one launch from the ncu capture recorded in
-    profiles/traffic.json, or None when the kernel source has changed since."""
-    import hashlib
+    profiles/traffic.json, or None when the kernel's code (its sources without
+    comments) has changed since the capture."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             rec = json.load(f).get(workload)
         if not rec:
             return None
-        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
-            if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
-                return None
+        if code_digest(rec["sources"]) != rec["code_digest"]:
+            return None
         return rec["traffic_bytes"]
     except (OSError, ValueError, KeyError):
         return None

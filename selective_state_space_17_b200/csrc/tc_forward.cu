@@ -8,7 +8,8 @@
 //   MMA1    S  = C B^T                                  (128 x 128, K = N)  TMEM
 //   states  s  = B^T (w o X),  w_j = exp(cs_end - cs_j) dt_j  (N x 64, K = 128) TMEM
 //   mask    S~_ij = S_ij exp(cs_i - cs_j) dt_j (j <= i), plus D_h on the diagonal,
-//           in registers, written as bf16 over the tile's B in shared memory
+//           in registers, written back as bf16 pairs over S in TMEM (the A
+//           operand of MMA2)
 //   MMA2    Yd = S~ X                                   (128 x 64, K = 128) TMEM
 //   MMA3    Ys = C h_prev^T                             (128 x 64, K = N)   TMEM
 //   output  y_i = Yd_i + exp(cs_i) Ys_i (bf16, round to nearest even)
@@ -25,14 +26,21 @@
 // exp(cs_i - cs_j) = exp(cs_i - cs_a) * exp(cs_a - cs_j), both factors <= 1,
 // so only the block on the diagonal needs one exponential per element.
 //
-// Schedule. Each (batch row, head) is a chain of tiles; chains are cut into
-// segments of `seg_len` tiles. A work item is one segment of one chain, and
+// Schedule. Each (batch row, head) is a chain of tiles (a head of P = 64m
+// channels is m chains of 64 channels); chains are cut into segments of
+// `seg_len` tiles. A work item is one segment of one chain, and
 // items are numbered segment-major, so an item's predecessor (the previous
 // segment of the same chain) is numbered `chains` earlier. One persistent CTA
 // per SM takes items blockIdx.x, blockIdx.x + gridDim.x, ... and walks each
 // item's tiles in order with the state h kept in registers; only at a segment
 // boundary does h travel through the workspace (a two-slot fp32 ring per
 // chain, published with a release flag and read after a bounded acquire poll).
+// Few chains cut into many segments would wait on each other's states one
+// after another; they run segment-parallel instead, in three launches: every
+// segment's local end state and total decay (mode 1, the state path only), a
+// scan over the segments (segment_scan_kernel), then every segment's outputs
+// from its scanned entering state (mode 2). A state dim above 128 runs as two
+// passes over the state columns, the second adding into y.
 //
 // Warp roles inside the CTA (416 threads), linked by full/empty mbarrier rings
 // whose waits sleep rather than spin:
@@ -48,7 +56,8 @@
 //   warps 3, 12   tile prologue: cumsum, column factors, w o X
 //   warps 4-7     mask S -> S~, in place in TMEM
 //   warps 8-11    h_prev -> bf16 operand, state update, epilogue through a
-//                 TMA store, look-back and segment publication
+//                 TMA store (a TMA reduce-add in a second pass over the
+//                 state columns), look-back and segment publication
 //
 // A chunk of 256 tokens is evaluated as two 128-token tiles: its quadratic
 // form split into 2 x 2 blocks, the diagonal blocks computed directly and the
@@ -70,8 +79,8 @@ namespace {
 using namespace sm100;
 
 constexpr int kT = 128;   // tokens per tile
-constexpr int kP = 64;    // head dim on this path
-constexpr int kN = 128;   // state dim of the tiles; a smaller N is zero-padded up to it
+constexpr int kP = 64;    // channels of a tile's head (a head of P = 64m runs as m of them)
+constexpr int kN = 128;   // state dim of a pass; a smaller N is zero-padded, a larger one takes two passes
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint64_t kMbarLimit = 1ull << 22;  // polls; each wait is also capped at ~2 s
 
