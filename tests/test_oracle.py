@@ -250,6 +250,43 @@ def test_group_broadcast_matches_per_head_copies(oracle):
     assert _rel(y, y2) < 1e-15 and _rel(fs, fs2) < 1e-15
 
 
+def test_state_columns_split_into_independent_problems(oracle):
+    """Each column n of the state evolves on its own (h_t = a_t h_{t-1} +
+    dt_t x_t B_tᵀ acts column by column) and y_t = h_t C_t sums over columns, so
+    a run over all N columns equals the sum of runs over two column blocks (D
+    counted once) and its final state is their concatenation. The tensor-core
+    path takes state dims above 128 this way, in two passes."""
+    rng = np.random.default_rng(21)
+    x, dt, A, Bm, Cm, D = _rand(rng, 2, 40, 4, 3, 2, 10)
+    init = rng.standard_normal((2, 4, 3, 10))
+    y, fs = oracle.forward(x, dt, A, Bm, Cm, D, init_state=init)
+    lo, hi = slice(0, 6), slice(6, 10)
+    c = np.ascontiguousarray
+    y1, f1 = oracle.forward(x, dt, A, c(Bm[..., lo]), c(Cm[..., lo]), D, init_state=c(init[..., lo]))
+    y2, f2 = oracle.forward(x, dt, A, c(Bm[..., hi]), c(Cm[..., hi]), None, init_state=c(init[..., hi]))
+    assert _rel(y1 + y2, y) < 1e-12
+    assert _rel(np.concatenate([f1, f2], axis=-1), fs) < 1e-15
+
+
+def test_wide_head_splits_into_narrower_heads(oracle):
+    """Each row p of the state evolves on its own, so a head of P = m q channels
+    equals m heads of q channels that share its dt, A and D: x, y [B, L, H, P]
+    and the states [B, H, P, N] read as [B, L, H m, q] and [B, H m, q, N]. The
+    tensor-core path runs P = 64m this way."""
+    rng = np.random.default_rng(22)
+    Bsz, L, H, P, G, N, m = 2, 30, 4, 6, 2, 5, 2
+    x, dt, A, Bm, Cm, D = _rand(rng, Bsz, L, H, P, G, N)
+    init = rng.standard_normal((Bsz, H, P, N))
+    y, fs = oracle.forward(x, dt, A, Bm, Cm, D, init_state=init)
+    q = P // m
+    xs = x.reshape(Bsz, L, H * m, q)
+    dts = np.ascontiguousarray(np.repeat(dt, m, axis=2))
+    ys, fss = oracle.forward(xs, dts, np.repeat(A, m), Bm, Cm, np.repeat(D, m),
+                             init_state=init.reshape(Bsz, H * m, q, N))
+    assert _rel(ys.reshape(Bsz, L, H, P), y) < 1e-15
+    assert _rel(fss.reshape(Bsz, H, P, N), fs) < 1e-15
+
+
 # ------------------------------------------------------------------------- decode
 
 def test_step_from_zero_reproduces_forward(oracle):
