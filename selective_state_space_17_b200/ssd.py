@@ -86,15 +86,32 @@ def _stream_handle(stream) -> int:
     return stream.cuda_stream
 
 
-def _need(t, name, dtype=None, device=None):
+def _need(t, name, dtype=None, device=None, shape=None, cuda=True):
+    """Checks one tensor argument before anything reaches the library: a host
+    tensor handed to a device entry point (or the reverse) would otherwise
+    become a wild pointer inside a kernel."""
     if t is None:
         raise ValueError(f"{name} is required")
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor, got {type(t).__name__}")
+    if cuda and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (got one on {t.device})")
+    if not cuda and t.is_cuda:
+        raise ValueError(f"{name} must be a host tensor (got one on {t.device})")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if device is not None and t.device != device:
-        raise ValueError(f"{name} must be on {device}")
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _dims4(x, name):
+    if x.dim() != 4:
+        raise ValueError(f"{name} must be [B, L, H, P], got shape {tuple(x.shape)}")
+    return tuple(x.shape)
 
 
 _ws_lock = threading.Lock()
@@ -105,10 +122,13 @@ def workspace_size(B, L, H, P, G, N, chunk, dtype_code) -> int:
     return int(lib.ssd_workspace_size(B, L, H, P, G, N, chunk, dtype_code))
 
 
-def _workspace(device, nbytes: int) -> torch.Tensor:
-    """A zero-filled workspace of at least nbytes, cached per device and stream
-    user. The library leaves its control words zeroed after each call."""
-    key = (device.index if device.index is not None else torch.cuda.current_device())
+def _workspace(device, nbytes: int, stream_handle: int) -> torch.Tensor:
+    """A zero-filled workspace of at least nbytes, cached per (device, stream):
+    calls on one stream are ordered and may share it (the library leaves its
+    control words zeroed after each call); calls on two streams may overlap on
+    the GPU, so each stream gets its own."""
+    dev_index = device.index if device.index is not None else torch.cuda.current_device()
+    key = (dev_index, stream_handle)
     with _ws_lock:
         ws = _ws_cache.get(key)
         if ws is None or ws.numel() < nbytes:
@@ -125,33 +145,39 @@ def forward(x, dt, A, Bm, Cm, D=None, chunk: int = 256, initial_state=None, y=No
     _need(x, "x")
     dev = x.device
     code = _dtype_code(x)
-    Bsz, L, H, P = x.shape
+    Bsz, L, H, P = _dims4(x, "x")
     _need(Bm, "Bm", x.dtype, dev)
-    _need(Cm, "Cm", x.dtype, dev)
+    if Bm.dim() != 4:
+        raise ValueError(f"Bm must be [B, L, G, N], got shape {tuple(Bm.shape)}")
     G, N = Bm.shape[2], Bm.shape[3]
-    if tuple(Bm.shape) != (Bsz, L, G, N) or tuple(Cm.shape) != tuple(Bm.shape):
-        raise ValueError("Bm and Cm must be [B, L, G, N]")
-    _need(dt, "dt", torch.float32, dev)
-    _need(A, "A", torch.float32, dev)
-    if tuple(dt.shape) != (Bsz, L, H) or tuple(A.shape) != (H,):
-        raise ValueError("dt must be [B, L, H] and A [H]")
+    _need(Bm, "Bm", shape=(Bsz, L, G, N))
+    _need(Cm, "Cm", x.dtype, dev, (Bsz, L, G, N))
+    _need(dt, "dt", torch.float32, dev, (Bsz, L, H))
+    _need(A, "A", torch.float32, dev, (H,))
     if D is not None:
-        _need(D, "D", torch.float32, dev)
+        _need(D, "D", torch.float32, dev, (H,))
     if initial_state is not None:
-        _need(initial_state, "initial_state", torch.float32, dev)
+        _need(initial_state, "initial_state", torch.float32, dev, (Bsz, H, P, N))
     if y is None:
         y = torch.empty_like(x)
+    else:
+        _need(y, "y", x.dtype, dev, (Bsz, L, H, P))
     if final_state is None and return_final_state:
         final_state = torch.empty((Bsz, H, P, N), dtype=torch.float32, device=dev)
+    elif final_state is not None:
+        _need(final_state, "final_state", torch.float32, dev, (Bsz, H, P, N))
     nbytes = workspace_size(Bsz, L, H, P, G, N, chunk, code)
     if nbytes == 0:
         raise SSDError(1, "ssd_workspace_size")
+    sh = _stream_handle(stream)
     if workspace is None:
-        workspace = _workspace(dev, nbytes)
+        workspace = _workspace(dev, nbytes, sh)
+    else:
+        _need(workspace, "workspace", device=dev)
     rc = lib.ssd_forward(_ptr(x), _ptr(dt), _ptr(A), _ptr(Bm), _ptr(Cm), _ptr(D),
                          _ptr(initial_state), _ptr(y), _ptr(final_state),
                          Bsz, L, H, P, G, N, chunk, code, _ptr(workspace),
-                         workspace.numel() * workspace.element_size(), _stream_handle(stream))
+                         workspace.numel() * workspace.element_size(), sh)
     _check(rc, "ssd_forward")
     return y, final_state
 
@@ -177,16 +203,36 @@ def forward_host(x, dt, A, Bm, Cm, D, y, final_state=None, initial_state=None, c
     copies the inputs in, runs the forward, copies y / final_state out and
     synchronises the stream. Shapes as ``forward``; y (and final_state) are
     caller-provided host tensors that receive the result."""
+    _need(x, "x", cuda=False)
     code = _dtype_code(x)
-    Bsz, L, H, P = x.shape
+    Bsz, L, H, P = _dims4(x, "x")
+    _need(Bm, "Bm", x.dtype, cuda=False)
+    if Bm.dim() != 4:
+        raise ValueError(f"Bm must be [B, L, G, N], got shape {tuple(Bm.shape)}")
     G, N = Bm.shape[2], Bm.shape[3]
+    _need(Bm, "Bm", shape=(Bsz, L, G, N), cuda=False)
+    _need(Cm, "Cm", x.dtype, shape=(Bsz, L, G, N), cuda=False)
+    _need(dt, "dt", torch.float32, shape=(Bsz, L, H), cuda=False)
+    _need(A, "A", torch.float32, shape=(H,), cuda=False)
+    if D is not None:
+        _need(D, "D", torch.float32, shape=(H,), cuda=False)
+    if initial_state is not None:
+        _need(initial_state, "initial_state", torch.float32, shape=(Bsz, H, P, N), cuda=False)
+    _need(y, "y", x.dtype, shape=(Bsz, L, H, P), cuda=False)
+    if final_state is not None:
+        _need(final_state, "final_state", torch.float32, shape=(Bsz, H, P, N), cuda=False)
     need = forward_host_buffer_size(Bsz, L, H, P, G, N, chunk, code)
+    if need == 0:
+        raise SSDError(1, "ssd_forward_host_buffer_size")
     if device_buffer is None:
         device_buffer = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    else:
+        _need(device_buffer, "device_buffer")
     rc = lib.ssd_forward_host(_ptr(x), _ptr(dt), _ptr(A), _ptr(Bm), _ptr(Cm), _ptr(D),
                               _ptr(initial_state), _ptr(y), _ptr(final_state),
                               Bsz, L, H, P, G, N, chunk, code, _ptr(device_buffer),
-                              device_buffer.numel(), _stream_handle(stream))
+                              device_buffer.numel() * device_buffer.element_size(),
+                              _stream_handle(stream))
     _check(rc, "ssd_forward_host")
     return y, final_state
 
@@ -194,14 +240,26 @@ def forward_host(x, dt, A, Bm, Cm, D, y, final_state=None, initial_state=None, c
 def step(x, dt, A, Bm, Cm, D, state, y=None, stream=None):
     """One decode step; ``state`` [B,H,P,N] f32 is updated in place. Returns y."""
     _need(x, "x")
+    dev = x.device
     code = _dtype_code(x)
+    if x.dim() != 3:
+        raise ValueError(f"x must be [B, H, P], got shape {tuple(x.shape)}")
     Bsz, H, P = x.shape
+    _need(Bm, "Bm", x.dtype, dev)
+    if Bm.dim() != 3:
+        raise ValueError(f"Bm must be [B, G, N], got shape {tuple(Bm.shape)}")
     G, N = Bm.shape[1], Bm.shape[2]
-    _need(Bm, "Bm", x.dtype, x.device)
-    _need(Cm, "Cm", x.dtype, x.device)
-    _need(state, "state", torch.float32, x.device)
+    _need(Bm, "Bm", shape=(Bsz, G, N))
+    _need(Cm, "Cm", x.dtype, dev, (Bsz, G, N))
+    _need(dt, "dt", torch.float32, dev, (Bsz, H))
+    _need(A, "A", torch.float32, dev, (H,))
+    if D is not None:
+        _need(D, "D", torch.float32, dev, (H,))
+    _need(state, "state", torch.float32, dev, (Bsz, H, P, N))
     if y is None:
         y = torch.empty_like(x)
+    else:
+        _need(y, "y", x.dtype, dev, (Bsz, H, P))
     rc = lib.ssd_step(_ptr(x), _ptr(dt), _ptr(A), _ptr(Bm), _ptr(Cm), _ptr(D), _ptr(state),
                       _ptr(y), Bsz, H, P, G, N, code, _stream_handle(stream))
     _check(rc, "ssd_step")
