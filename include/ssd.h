@@ -60,7 +60,8 @@ typedef enum {
 
 typedef enum {
     SSD_F32 = 0,   /* x, Bm, Cm, y in fp32: SIMT fp32 path (|rel err| ~1e-6) */
-    SSD_BF16 = 1   /* x, Bm, Cm, y in bf16: tensor-core path, fp32 accumulate */
+    SSD_BF16 = 1   /* x, Bm, Cm, y in bf16, fp32 accumulate: tensor-core path for the
+                      sizes ssd_forward lists, SIMT path otherwise */
 } ssd_dtype;
 
 /* Human-readable name of a status code (static string, never NULL). */
