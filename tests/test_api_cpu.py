@@ -61,6 +61,41 @@ def test_kernel_count_query(lib):
     assert lib.ssd_forward_kernel_count(1, 64, 2, 8, 1, 8, 16, 0) == 3
 
 
+def test_workspace_size_formula(lib):
+    """Single pass: 256 B of control words, one 4-byte flag per chain rounded up
+    to 256 B, and a two-slot [128][64] fp32 state ring per chain, where a chain
+    is one 64-channel head slice of one batch row (M = B*H*P/64); the query adds
+    256 bytes of slack."""
+    def single(M):
+        return 256 + (4 * M + 255) // 256 * 256 + M * 2 * 64 * 128 * 4 + 256
+    assert lib.ssd_workspace_size(4, 4096, 80, 64, 1, 128, 256, 1) == single(4 * 80)
+    assert lib.ssd_workspace_size(8, 2048, 32, 64, 1, 128, 256, 1) == single(8 * 32)
+    assert lib.ssd_workspace_size(2, 8192, 64, 64, 8, 256, 256, 1) == single(2 * 64)  # two passes share it
+    assert lib.ssd_workspace_size(2, 512, 4, 128, 2, 128, 128, 1) == single(2 * 4 * 2)  # wide heads
+
+
+def test_segment_parallel_workspace_adds_per_segment_states(lib):
+    # long context: 32 chains of 512 tiles; with 148 SMs (the value assumed
+    # without a GPU) each chain is cut into 37 segments of 14 tiles
+    M, nseg = 32, 37
+    base = 256 + 256 + M * 2 * 64 * 128 * 4 + 256  # control, flags, ring, slack
+    slot = 64 * 128 * 4
+    extra = M * nseg * slot + (4 * M * nseg + 255) // 256 * 256 + M * nseg * slot
+    assert lib.ssd_forward_path(1, 65536, 32, 64, 1, 128, 256, 1) == 3
+    assert lib.ssd_forward_kernel_count(1, 65536, 32, 64, 1, 128, 256, 1) == 3
+    assert lib.ssd_workspace_size(1, 65536, 32, 64, 1, 128, 256, 1) == base + extra
+
+
+def test_benchmark_workloads_take_the_tensor_core_path(lib):
+    assert lib.ssd_forward_path(4, 4096, 80, 64, 1, 128, 256, 1) == 2      # 2.7B layer
+    assert lib.ssd_forward_kernel_count(4, 4096, 80, 64, 1, 128, 256, 1) == 1
+    assert lib.ssd_forward_path(8, 2048, 32, 64, 1, 128, 256, 1) == 2      # 370M layer
+    for N in (16, 32, 64, 128, 256):                                       # sweep
+        for Q in (128, 256):
+            assert lib.ssd_forward_path(2, 8192, 64, 64, 8, N, Q, 1) == 2
+            assert lib.ssd_forward_kernel_count(2, 8192, 64, 64, 8, N, Q, 1) == (2 if N > 128 else 1)
+
+
 def test_status_strings(lib):
     for code in range(7):
         s = lib.ssd_status_string(code).decode()
