@@ -211,7 +211,18 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(rows)}
 
 
-def time_oracle_sample(w: gen.Workload, inp, heads: int, min_seconds: float):
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def time_oracle_sample(w: gen.Workload, inp, heads: int, min_seconds: float, threads=None):
     """Run the fp64 oracle on batch row 0, the first `heads` heads (their
     groups whole), full sequence; repeat until min_seconds. Returns
     (Mtokens/s-equivalent, threads, sample description, seconds)."""
@@ -221,7 +232,7 @@ def time_oracle_sample(w: gen.Workload, inp, heads: int, min_seconds: float):
         heads = max(hpg, (heads // hpg) * hpg)
     heads = min(heads, w.H)
     x, dt, A, Bm, Cm, D = inp.f64(0, 1, heads=(0, heads))
-    threads = min(oracle.default_threads(), heads)
+    threads = min(threads or oracle.default_threads(), heads)
     reps, t0 = 0, time.perf_counter()
     while True:
         oracle.forward(x, dt, A, Bm, Cm, D, nthreads=threads)
@@ -331,11 +342,16 @@ def run_ours(args):
     per_step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     ms, _ = combine_ranks(statistics.mean(per_step_ms), w.tokens, world, dist, dev)
     decode = time_decode(ssd, dev, flush, args.warmup, args.steps, world, dist)
+    workloads = None
+    if not args.no_workloads:
+        workloads = [time_workload(ssd, v, dev, flush, 3, args.steps, world, dist)
+                     for v in secondary_workloads() if v.name != w.name]
+        torch.cuda.empty_cache()
 
     # end to end through the host-buffer entry point: H2D inputs, forward, D2H y + state
     if args.no_e2e:
         return _report(args, w, rank, world, ms, per_step_ms, clk, inp, None, host, ssd, code, dist,
-                       decode)
+                       decode, workloads)
     pin = {k: v.pin_memory() for k, v in host.items()}
     y_host = torch.empty_like(host["x"]).pin_memory()
     fs_host = torch.empty((w.B, w.H, w.P, w.N), dtype=torch.float32).pin_memory()
@@ -359,44 +375,115 @@ def run_ours(args):
     barrier()
     e2e_ms, _ = combine_ranks(e_start.elapsed_time(e_end) / e2e_steps, w.tokens, world, dist, dev)
     return _report(args, w, rank, world, ms, per_step_ms, clk, inp, e2e_ms, host, ssd, code, dist,
-                   decode)
+                   decode, workloads)
 
 
-def time_decode(ssd, dev, flush, warmup, steps, world, dist):
+def device_inputs(w: gen.Workload, seed: int, dev):
+    """Inputs of the recipe in inputs.make_inputs (x ~ N(0,1); dt = exp(U[ln 1e-3,
+    ln 1e-1]); A = -exp(U[0, ln 16]); Bm, Cm ~ N(0,1)/sqrt(N); D ~ N(0,1); the
+    a = 1 and a = 0.99 kinds with dt = 1), drawn on the GPU with torch's seeded
+    generator and rounded once to the I/O dtype. Used for the secondary
+    workloads, whose timing needs their shapes and distributions; the headline
+    workload uses the numpy sample the parity tests check."""
+    import torch
+    g = torch.Generator(device=dev).manual_seed(1000 + seed)
+    io = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    x = torch.randn(w.B, w.L, w.H, w.P, device=dev, generator=g).to(io)
+    dt = torch.exp(torch.empty(w.B, w.L, w.H, device=dev).uniform_(
+        float(np.log(1e-3)), float(np.log(1e-1)), generator=g))
+    A = -torch.exp(torch.empty(w.H, device=dev).uniform_(0.0, float(np.log(16.0)), generator=g))
+    Bm = (torch.randn(w.B, w.L, w.G, w.N, device=dev, generator=g) / w.N ** 0.5).to(io)
+    Cm = (torch.randn(w.B, w.L, w.G, w.N, device=dev, generator=g) / w.N ** 0.5).to(io)
+    D = torch.randn(w.H, device=dev, generator=g)
+    if w.kind in ("linear_attention", "retnet"):
+        dt.fill_(1.0)
+        A.fill_(0.0 if w.kind == "linear_attention" else float(np.log(0.99)))
+    return dict(x=x, dt=dt, A=A, Bm=Bm, Cm=Cm, D=D)
+
+
+def secondary_workloads():
+    """The other configurations of the layer: the 370M-shaped layer, the long
+    context, the state-size / grouping sweep and its a = 1 and a = 0.99 runs."""
+    ws = [gen.LAYER_370M, gen.LONG_CONTEXT] + gen.sweep_workloads()
+    ws += [v for v in gen.sweep_workloads(("linear_attention", "retnet")) if " N128 Q256" in v.name]
+    return ws
+
+
+def time_workload(ssd, w: gen.Workload, dev, flush, warmup, steps, world, dist):
+    """One secondary workload, timed like the headline: L2 flushed between steps
+    outside the events, the mean of `steps` steps, max over ranks."""
+    import torch
+    d = device_inputs(w, 0, dev)
+    code = ssd.SSD_BF16 if w.dtype == "bf16" else ssd.SSD_F32
+    y = torch.empty_like(d["x"])
+    fs = torch.empty((w.B, w.H, w.P, w.N), dtype=torch.float32, device=dev)
+    ws = torch.zeros(ssd.workspace_size(w.B, w.L, w.H, w.P, w.G, w.N, w.chunk, code),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ssd.forward(d["x"], d["dt"], d["A"], d["Bm"], d["Cm"], d["D"], chunk=w.chunk, y=y,
+                    final_state=fs, workspace=ws, stream=stream)
+
+    for _ in range(warmup):
+        flush()
+        step()
+    times = []
+    for _ in range(steps):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        times.append((e0, e1))
+    ssd.poll_status(stream)
+    ms, value = combine_ranks(statistics.mean(a.elapsed_time(b) for a, b in times), w.tokens,
+                              world, dist, dev)
+    hbm_peak, tc_peak, _ = measured_peaks()
+    t_roof = max(compulsory_bytes(w) / (hbm_peak * 1e9), algorithmic_flops(w) / (tc_peak * 1e12))
+    return {"workload": w.name, "ms_per_step": ms, "value": value, "unit": UNIT,
+            "roofline_frac": t_roof * 1e3 / ms,
+            "path": ssd.forward_path(w.B, w.L, w.H, w.P, w.G, w.N, w.chunk, code),
+            "launches_per_step": ssd.kernel_count(w.B, w.L, w.H, w.P, w.G, w.N, w.chunk, code)}
+
+
+def time_decode(ssd, dev, flush, warmup, steps, world, dist, rotate=4):
     """ssd_step on the decode workload (one token for each of B sequences from a
-    random fp32 state), L2 flushed between steps outside the events."""
+    random fp32 state). The steps run back to back over `rotate` independent
+    states (several layers' worth, 4 x 67 MB, twice the L2), all timed by one
+    pair of events: each step's state write-back is evicted, and so paid for,
+    inside the timed region (a flush between steps would pay it outside)."""
     import torch
     d = gen.DECODE
     s = gen.make_step_inputs(d["B"], d["H"], d["P"], d["G"], d["N"], d["dtype"], seed=5)
     io = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
     x, Bm, Cm = io(s.x), io(s.Bm), io(s.Cm)
     dt, A, D = (torch.from_numpy(v).to(dev) for v in (s.dt, s.A, s.D))
-    state = torch.from_numpy(s.state).to(dev)
+    states = [torch.from_numpy(s.state).to(dev) for _ in range(rotate)]
     y = torch.empty_like(x)
     stream = torch.cuda.current_stream()
-    for _ in range(warmup):
-        flush()
-        ssd.step(x, dt, A, Bm, Cm, D, state, y=y, stream=stream)
-    times = []
-    for _ in range(steps):
-        flush()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        ssd.step(x, dt, A, Bm, Cm, D, state, y=y, stream=stream)
-        e1.record(stream)
-        times.append((e0, e1))
+    n = max(steps, 4 * rotate)
+    for i in range(max(warmup, rotate)):
+        ssd.step(x, dt, A, Bm, Cm, D, states[i % rotate], y=y, stream=stream)
+    flush()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(n):
+        ssd.step(x, dt, A, Bm, Cm, D, states[i % rotate], y=y, stream=stream)
+    e1.record(stream)
     ssd.poll_status(stream)
-    ms, _ = combine_ranks(statistics.mean(a.elapsed_time(b) for a, b in times), d["B"], world,
-                          dist, dev)
+    ms, _ = combine_ranks(e0.elapsed_time(e1) / n, d["B"], world, dist, dev)
     nbytes = (2 * d["B"] * d["H"] * d["P"] * d["N"] * 4 + 2 * d["B"] * d["H"] * d["P"] * 2
               + d["B"] * d["H"] * 4 + 2 * d["B"] * d["G"] * d["N"] * 2 + 2 * d["H"] * 4)
     return {"workload": d["name"], "ms_per_step": ms,
             "value": d["B"] * world / (ms / 1e3) / 1e6, "unit": "Mtokens/s",
-            "algorithmic_bytes": nbytes, "achieved_gbs": nbytes / (ms / 1e3) / 1e9}
+            "algorithmic_bytes": nbytes, "achieved_gbs": nbytes / (ms / 1e3) / 1e9,
+            "timing": f"{n} steps back to back over {rotate} independent states "
+                      f"({rotate * d['B'] * d['H'] * d['P'] * d['N'] * 4 >> 20} MiB), one event pair"}
 
 
 def _report(args, w, rank, world, ms, per_step_ms, clk, inp, e2e_ms, host, ssd, code, dist,
-            decode=None):
+            decode=None, workloads=None):
     tokens_all = w.tokens * world
     value = tokens_all / (ms / 1e3) / 1e6
     h2d = sum(v.numel() * v.element_size() for v in host.values())
@@ -446,12 +533,17 @@ def _report(args, w, rank, world, ms, per_step_ms, clk, inp, e2e_ms, host, ssd, 
                 peak=hbm_peak, peak_unit="GB/s"),
             "per_step_ms": {"min": min(per_step_ms), "median": statistics.median(per_step_ms),
                             "max": max(per_step_ms)},
+            "workloads": workloads,
         }
         if world == 1 and not args.no_cpu_baseline:
             v, threads, sample, el = time_oracle_sample(w, inp, heads=16, min_seconds=10.0)
+            v1, _, sample1, el1 = time_oracle_sample(w, inp, heads=1, min_seconds=5.0, threads=1)
             result["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads,
                                       "kind": "oracle", "sample": sample,
-                                      "seconds": round(el, 2)}
+                                      "seconds": round(el, 2), "cpu_model": cpu_model(),
+                                      "nproc": os.cpu_count(),
+                                      "one_core": {"value": v1, "unit": UNIT, "cores": 1,
+                                                   "sample": sample1, "seconds": round(el1, 2)}}
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -470,6 +562,8 @@ def main():
                     help="skip the oracle timing on the host cores")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer end-to-end timing (used for profiling runs)")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the secondary workloads (370M, long context, sweep)")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="2.7b",
                     help="layer configuration (default: the 2.7B-shaped layer)")
     args = ap.parse_args()

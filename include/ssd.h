@@ -68,13 +68,14 @@ typedef enum {
 const char* ssd_status_string(ssd_status status);
 
 /* Bytes of device workspace ssd_forward needs for these sizes (0 if the sizes
- * are invalid). On the tensor-core path the size depends on the current
+ * are invalid). On the tensor-core paths the size depends on the current
  * device's SM count, which decides how each (batch, head) chain is cut into
- * segments; ask on the device that will run the call. The workspace must be
- * zero-filled once before its first use (e.g. cudaMemset); every call leaves
- * its control words zeroed again, so a workspace can be reused by later calls
- * on the same stream without clearing. Two calls that run concurrently must
- * not share one workspace. */
+ * segments; ask on the device that will run the call. The workspace needs no
+ * clearing, neither before its first use nor between calls: the control words
+ * a call keeps there (look-back flags, a work ticket counter) carry a tag of
+ * that call, so leftovers of any earlier call, of any path or size, read as
+ * unwritten. Calls ordered on one stream may therefore share a workspace; two
+ * calls that run concurrently must not. */
 size_t ssd_workspace_size(int B, int L, int H, int P, int G, int N, int chunk, ssd_dtype dtype);
 
 /*
@@ -92,17 +93,31 @@ size_t ssd_workspace_size(int B, int L, int H, int P, int G, int N, int chunk, s
  *   Sizes: B, L >= 0 (B*L == 0 is a no-op apart from final_state =
  *   initial_state or 0), H >= 1, G >= 1, H % G == 0, P in [1, 256],
  *   N in [1, 256]. All pointers 16-byte aligned.
- *   The tensor-core path is taken for bf16 with P a multiple of 64 (a head of
- *   P = 64m channels runs as m heads of 64 channels sharing dt, A and D: the
- *   rows of the P x N state evolve independently), N a multiple of 8
+ *   The tensor-core paths are taken for bf16 with P a multiple of 64 (a head
+ *   of P = 64m channels runs as m heads of 64 channels sharing dt, A and D:
+ *   the rows of the P x N state evolve independently), N a multiple of 8
  *   with 8 <= N <= 256, and chunk in {64, 128, 256}; other valid sizes run
- *   the SIMT path. The tensor-core path evaluates the chunked form on
+ *   the SIMT path. Both tensor-core kernels evaluate the chunked form on
  *   128-token tiles whatever `chunk` is (the result does not depend on the
- *   chunk length beyond rounding). With N > 128 it runs two passes over the
- *   state columns (n < 128, then the rest; each state column evolves on its
- *   own and y is a sum over columns): the first stores y with the D term,
- *   the second adds its share into y in L2 (a bf16 add, so y is rounded
- *   twice), and each writes its columns of final_state.
+ *   chunk length beyond rounding):
+ *   - the head-group kernel (N <= 128, and enough (batch, head pair) chains
+ *     to fill the GPU) takes two heads of one B/C group through each tile,
+ *     sharing C B^T between them ("Mamba-2", section "Mamba-2 block", item
+ *     2). Where a tile's total decay allows it, the decay mask is applied as
+ *     a row and a column scaling around a reference point of the tile (the
+ *     mask is a product of per-token decays); tiles of larger decay take an
+ *     exact per-head form. Segments of a chain are handed to CTAs in order
+ *     from a ticket counter, so a segment only waits on one that a running
+ *     CTA already holds.
+ *   - the per-head kernel takes the other sizes. With N > 128 it runs two
+ *     passes over the state columns (n < 128, then the rest; each state column
+ *     evolves on its own and y is a sum over columns): the first stores y with
+ *     the D term, the second adds its share into y in L2 (a bf16 add, so y is
+ *     rounded twice), and each writes its columns of final_state. It hands its
+ *     segments to CTAs statically and assumes every CTA of its grid (one per
+ *     SM) is resident at once: if other work keeps some SMs busy for seconds
+ *     (another stream, MPS), its bounded look-back waits give up and the call
+ *     reports SSD_ERR_TIMEOUT through ssd_poll_status() with undefined results.
  */
 ssd_status ssd_forward(const void* x, const float* dt, const float* A, const void* Bm,
                        const void* Cm, const float* D, const float* initial_state, void* y,
@@ -114,10 +129,12 @@ ssd_status ssd_forward(const void* x, const float* dt, const float* A, const voi
  * ssd_forward_noalloc — the forward pass for callers that cannot allocate
  * device memory. The pages describe no such entry point; it is a convenience
  * of this library. It takes the same arguments as ssd_forward without the
- * workspace: its scratch (look-back control words and the per-head state
- * ring, with M = B*H*P/64: 256 + 4*M rounded to 256, + 2*M*64*128*4 bytes) lives in a fixed
- * 24 MiB device array inside the library, which every GPU that loads the
- * library holds until the process exits. Only the tensor-core sizes are
+ * workspace and runs the per-head tensor-core kernel: its scratch (look-back
+ * flags and the per-head state ring, with M = B*H*P/64: 256 + 8*M rounded to
+ * 256, + 2*M*64*128*4 bytes) lives in a fixed 24 MiB device array inside the
+ * library, which every GPU that loads the library holds until the process
+ * exits. Nothing in the array needs clearing between calls (the flags carry
+ * a tag of the call that wrote them). Only the tensor-core sizes are
  * handled (bf16, P a multiple of 64, N a multiple of 8 up to 256, chunk 64, 128 or 256,
  * B*L > 0); other sizes return SSD_ERR_UNSUPPORTED, and sizes whose scratch
  * exceeds the array (M > 383; or, in the segment-parallel form, the two
@@ -136,9 +153,14 @@ ssd_status ssd_forward_noalloc(const void* x, const float* dt, const float* A, c
 /*
  * ssd_forward_host — the same forward pass on HOST buffers (pinned memory
  * gives asynchronous copies). Copies the inputs into `device_buffer`, runs
- * ssd_forward on `stream`, copies y (and final_state if non-NULL) back, and
- * synchronises `stream` before returning. `device_buffer` must hold at least
- * ssd_forward_host_buffer_size() bytes and be zero-filled before first use.
+ * the forward pass, copies y (and final_state if non-NULL) back, and
+ * synchronises `stream` before returning. The batch runs in up to four slices
+ * of rows on two internal streams of the library (created on the first call
+ * on a device, after the work already queued on `stream`), so that one
+ * slice's copies overlap another's forward pass and the two copy directions
+ * overlap each other. `device_buffer` must hold at least
+ * ssd_forward_host_buffer_size() bytes (the tensors plus one workspace per
+ * internal stream); it needs no clearing.
  */
 size_t ssd_forward_host_buffer_size(int B, int L, int H, int P, int G, int N, int chunk,
                                     ssd_dtype dtype);
@@ -170,10 +192,11 @@ int ssd_forward_kernel_count(int B, int L, int H, int P, int G, int N, int chunk
                              ssd_dtype dtype);
 
 /* Which path one ssd_forward call with these sizes takes: 0 if the sizes are
- * invalid or there are no tokens, 1 the SIMT path, 2 the tensor-core single
- * pass, 3 the tensor-core segment-parallel form (fewer (batch, head) chains
- * than half the SMs, each cut into eight or more segments: few chains on long
- * sequences). Host-side query; it
+ * invalid or there are no tokens, 1 the SIMT path, 2 the per-head tensor-core
+ * kernel's single pass, 3 its segment-parallel form (fewer (batch, head)
+ * chains than half the SMs, each cut into eight or more segments: few chains
+ * on long sequences), 4 the head-group tensor-core kernel (two heads of one
+ * B/C group per tile; N <= 128 with enough chains). Host-side query; it
  * reads the current device's SM count and launches nothing. */
 int ssd_forward_path(int B, int L, int H, int P, int G, int N, int chunk, ssd_dtype dtype);
 
@@ -193,6 +216,13 @@ void ssd_set_wait_limit(uint64_t iterations);
  * ssd_poll_status(). Results of such calls are garbage. 0 restores normal
  * operation. */
 void ssd_set_fault_injection(int skip_publish);
+
+/* Test hook: which tensor-core kernel ssd_forward uses when both handle the
+ * sizes. 0 (the default) picks the faster for the sizes, 1 forces the
+ * per-head kernel, 2 the head-group kernel (bf16, P a multiple of 64,
+ * N <= 128). Other values restore 0. ssd_workspace_size() already covers
+ * either kernel. */
+void ssd_set_forward_variant(int variant);
 
 #ifdef __cplusplus
 }

@@ -46,7 +46,34 @@ struct LaunchCtx {
     unsigned int* status;        // device status word
     unsigned long long wait_limit;  // iterations of a bounded device wait
     int num_sms;
+    // Tag of this call, never 0. The control words a call keeps in its
+    // workspace (look-back flags, ticket counter) are 64-bit values whose high
+    // half is the tag of the call that wrote them, so whatever an earlier call
+    // of any path or size left there reads as not yet written: a workspace
+    // needs no clearing, before its first use or between calls.
+    uint32_t epoch;
 };
+
+// Control word of this call: (epoch, count).
+__host__ __device__ __forceinline__ unsigned long long tagged(uint32_t epoch, uint32_t count)
+{
+    return (static_cast<unsigned long long>(epoch) << 32) | count;
+}
+
+// Takes the next value of a per-call counter kept as a tagged word: the first
+// taker of a call finds another call's tag (or garbage) and restarts the count
+// at 0 for this call.
+__device__ __forceinline__ unsigned int take_ticket(unsigned long long* ctr, uint32_t epoch)
+{
+    unsigned long long cur = atomicAdd(ctr, 0ull);
+    for (;;) {
+        const bool mine = static_cast<uint32_t>(cur >> 32) == epoch;
+        const unsigned long long want = mine ? cur + 1ull : tagged(epoch, 1u);
+        const unsigned long long prev = atomicCAS(ctr, cur, want);
+        if (prev == cur) return mine ? static_cast<unsigned int>(cur) : 0u;
+        cur = prev;
+    }
+}
 
 }  // namespace ssd
 
@@ -88,6 +115,9 @@ cudaError_t simt_forward(const FwdArgs& a, void* workspace, const LaunchCtx& ctx
 // Device status word, stream and limits for a launch on the current device
 // (api.cu).
 ssd_status acquire_launch_ctx(cudaStream_t stream, LaunchCtx* ctx);
+
+// Size checks of every entry point: SSD_OK or the status to return (api.cu).
+ssd_status check_dims(int B, int L, int H, int P, int G, int N, int chunk, ssd_dtype dtype);
 
 // Decode step (step.cu).
 cudaError_t step_forward(const StepArgs& a, const LaunchCtx& ctx);

@@ -1,0 +1,1234 @@
+// grouped_forward.cu — tensor-core (tcgen05) forward of the SSD layer with the
+// heads of one B/C group processed together.
+//
+// "Mamba-2" (docsaid.org), section "Mamba-2 block", item 2: B and C are shared
+// by every head of a group, like keys and queries shared across the heads of
+// an attention layer. So for a 128-token tile the matrix S = C B^T is the same
+// for every head of the group, and only the decay mask and X differ per head.
+// This kernel takes KH heads of one group (KH = 2, or 1 when a group has an
+// odd number of heads) through each tile together.
+//
+// The decay of a tile. With cs the tile-local cumulative sum of dt * A in
+// log2 units (non-increasing, since dt >= 0 and A <= 0) and any reference
+// value c, the mask of the masked form factors into a row and a column term,
+//     2^(cs_i - cs_j) dt_j = 2^(cs_i - c) * (2^(c - cs_j) dt_j),
+// which turns the per-head masked product into one shared matrix tril(S)
+// times a per-head row-scaled X ("Mamba-2 SSD note" (0h-n0.github.io),
+// section "SSD layer: equivalence under the scalar constraint": the mask is a
+// product of decays, L_ij = a_i ... a_{j+1}). With c = cs_end / 2 every
+// factor lies in [2^(cs_end/2), 2^(-cs_end/2)], so while the tile's total
+// decay -cs_end stays below kHardLog2 nothing overflows or underflows. Per tile
+// ("scaled form"):
+//
+//   MMA1    S   = C B^T                              (128 x 128, K = N), TMEM
+//   mask    tril(S) as bf16 pairs, in place in TMEM (shared by the heads)
+//   X'      X'_h = diag(2^(c_h - cs_h,j) dt_h,j) X_h  (in place in shared memory)
+//   H'      H'_h = 2^(c_h) h_prev,h (bf16 operand), h <- 2^(c_h) h_prev,h in TMEM
+//   MMA3    Z   = C [H'_0 ... H'_KH-1]^T             (128 x 64 KH, K = N)
+//   MMA2    Z  += tril(S) [X'_0 ... X'_KH-1]         (128 x 64 KH, K = 128; A from TMEM)
+//   states  h  += B^T [X'_0 ... X'_KH-1]             (N x 64 KH, K = 128), so that
+//           h_new = 2^(cs_end - c) h (kept as a pending scalar)
+//   output  y_h,i = 2^(cs_h,i - c_h) Z_h,i + D_h x_h,i   (bf16, round to nearest even)
+//
+// A tile whose decay exceeds the bound ("exact form") keeps every factor <= 1:
+// X'_h = diag(2^(cs_end - cs_j) dt_j) X_h feeds the states only, H' = h_prev,
+// MMA3 writes C h_prev^T into Z, the output warps scale row i of Z by
+// 2^(cs_h,i) in place, and each head adds its own masked product
+// S~_h X_h with S~_h,ij = tril(S)_ij 2^(cs_h,i - cs_h,j) dt_h,j (built per head
+// in TMEM, X_h reloaded raw); then y = Z + D x. Both forms compute the chunked
+// algorithm of "Mamba-2", section "Half of each route": the quadratic form
+// inside a tile, the state across tiles (the composition of affine maps of
+// "Selective SSM guide" (auturnal.com), eq. (3)).
+//
+// Schedule. A chain is one batch row and one head group; it is cut into
+// segments of `seg_len` tiles, numbered segment-major, so a segment's
+// predecessor (the previous segment of its chain) is numbered `chains`
+// earlier. CTAs take segment numbers in order from a global ticket counter:
+// a CTA only waits on a segment that a running CTA took before it, so the
+// look-back cannot deadlock however many CTAs are resident. The state h of
+// the group's heads stays in TMEM from tile to tile; at a segment boundary it
+// travels through a per-chain slot in the workspace (release flag, bounded
+// acquire poll).
+//
+// Warp roles (416 threads), linked by full/empty mbarriers whose waits sleep
+// and are bounded (no named barriers, so a role that gives up cannot leave
+// another stuck):
+//   warp 0        producer: segment tickets, TMA loads of C, B (2 stages) and X
+//                 (KH heads, 2 stages); TMEM allocation
+//   warp 1        MMA stream A: MMA1 and states of each tile
+//   warp 2        MMA stream B: MMA3 and MMA2 (and the exact form's per-head
+//                 products, with the raw X reload)
+//   warps 3, 12   prologue, one head each: cumulative decay, tile record, X'
+//   warps 4-7     state and mask: h_prev -> H' and the scaled h, segment
+//                 hand-off and final state; then S -> tril(S) (exact form:
+//                 S~_h per head)
+//   warps 8-11    output: y = e Z + D x written to global memory (x loaded
+//                 while the tile's products run); the exact form's row
+//                 scaling of Z
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "grouped_forward.cuh"
+#include "sm100.cuh"
+#include "tma_map.cuh"
+
+namespace ssd {
+namespace grouped {
+namespace {
+
+using namespace sm100;
+
+constexpr int kT = 128;  // tokens per tile
+constexpr int kP = 64;   // channels of one head (a head of P = 64m is m of them)
+constexpr int kN = 128;  // largest state dim; a smaller N is zero-padded
+constexpr float kLog2e = 1.4426950408889634f;
+// Tiles whose decay (log2 units) exceeds this take the exact form: the scaled
+// form's factors then stay within 2^-72 .. 2^72.
+constexpr float kHardLog2 = 144.f;
+constexpr uint64_t kWaitNs = 2000000000ull;  // a role's wait on another gives up after ~2 s
+constexpr uint32_t kWaitPolls = 1u << 24;     // ... or after this many polls (each at most ~128 ns)
+
+constexpr int kThreads = 416;
+constexpr int kWarpProducer = 0;
+constexpr int kWarpMmaA = 1;
+constexpr int kWarpMmaB = 2;
+constexpr int kWarpPro0 = 3;   // prologue of head 0
+constexpr int kWarpPro1 = 12;  // prologue of head 1
+constexpr int kWgState = 4;    // warps 4..7
+constexpr int kWgOut = 8;      // warps 8..11
+constexpr int kSchedSlots = 4;
+constexpr int kPrefetch = 3;  // tiles ahead of the loads that the producer prefetches into L2
+constexpr int kSchedConsumers = 12;  // warps 1..12 read every ticket
+
+// TMEM columns (fp32, 128 lanes)
+constexpr uint32_t kColS = 0;    // 2 x 128: S, then tril(S) (bf16, cols 0-63) and S~_h (64-127)
+constexpr uint32_t kColH = 256;  // KH x 64: the states h, lane = state row n
+constexpr uint32_t kColZ = 384;  // KH x 64: Z, lane = token
+constexpr uint32_t kTmemCols = 512;
+
+constexpr uint32_t kHalf = 16384;  // one 128 x 64 bf16 block (a head's X, half of C or B)
+
+struct Rec {
+    float cs[2][kT];  // cumulative dt * A per head, log2 units
+    float cref[2];    // reference value c of the scaled form
+    float csend[2];   // cs of the tile's last token
+    int hard;         // exact form for this tile
+    int hardh[2];     // per head, before the two are combined
+    int pad[9];
+};
+static_assert(sizeof(Rec) == 1088, "record layout");
+
+struct Smem {
+    static constexpr uint32_t kC = 0;                    // 2 stages x 32 KB
+    static constexpr uint32_t kB = kC + 4 * kHalf;       // 2 stages x 32 KB
+    static constexpr uint32_t kX = kB + 4 * kHalf;       // 2 stages x KH x 16 KB (X, then X')
+    static constexpr uint32_t kHp = kX + 4 * kHalf;      // KH x 16 KB: H' (exact form: raw X)
+    static constexpr uint32_t kRec = kHp + 2 * kHalf;    // 2 records
+    static constexpr uint32_t kSched = kRec + 2 * sizeof(Rec);
+    static constexpr uint32_t kBars = kSched + 16;
+    static constexpr int kNumBars = 48;
+    static constexpr uint32_t kTmemPtr = kBars + kNumBars * 8;
+    static constexpr uint32_t kAbort = kTmemPtr + 4;
+    static constexpr uint32_t kBytes = kAbort + 4;
+};
+static_assert(Smem::kBytes <= 227 * 1024, "shared memory budget");
+
+enum Bar : int {
+    kFullCB = 0,      // 2 (tx)
+    kEmptyCB = 2,     // 2 (states, MMA3)
+    kFullX = 4,       // 2 (tx)
+    kEmptyX = 6,      // 2 (states, MMA2, the TMA store of y)
+    kXpFull = 8,      // 2 (four output warps)
+    kRecFull = 10,    // 2 (one per prologue warp)
+    kRecEmpty = 12,   // 2 (MMA B, four state and four output warps)
+    kSFull = 14,      // 2
+    kSFree = 16,      // 2
+    kTrilFull = 18,   // 2 (four state warps)
+    kHReady = 20,
+    kHpFull = 21,
+    kHpEmpty = 22,
+    kStatesDone = 23,
+    kZFull = 24,
+    kZEmpty = 25,     // four output warps
+    kM3Done = 26,     // exact form
+    kZScaled = 27,
+    kRawX = 28,
+    kSlotFull = 29,   // four state warps
+    kSlotFree = 30,
+    kSchedFull = 31,  // 4
+    kSchedEmpty = 35, // 4 (kSchedConsumers)
+    kDrainA = 39,
+    kDrainB = 40,
+    kHx = 41,         // the two prologue warps exchange their hard flags
+    kPub = 42,        // four state warps wrote a segment's end state
+    kYStaged = 43,    // four output warps wrote y over X'
+    kXRead = 44,      // 2: the states MMA of the tile in this X stage is done
+};
+
+uint32_t bar_count(int i, int kh)
+{
+    if (i == kEmptyCB || i == kEmptyCB + 1) return 2;
+    if (i == kEmptyX || i == kEmptyX + 1) return 3;
+    if (i == kRecFull || i == kRecFull + 1 || i == kHx) return kh;
+    if (i == kRecEmpty || i == kRecEmpty + 1) return 9;
+    if (i == kTrilFull || i == kTrilFull + 1 || i == kZEmpty || i == kSlotFull || i == kHReady ||
+        i == kHpFull || i == kZScaled || i == kPub || i == kXpFull || i == kXpFull + 1 || i == kYStaged)
+        return 4;
+    if (i >= kSchedEmpty && i < kSchedEmpty + kSchedSlots) return kSchedConsumers;
+    return 1;
+}
+
+struct GParams {
+    const float* dt;
+    const float* A;
+    const float* D;
+    const float* init;
+    const __nv_bfloat16* x;
+    __nv_bfloat16* y;
+    float* final_state;
+    unsigned long long* ctrl;   // [0] next ticket (tagged with the call's epoch)
+    unsigned long long* flags;  // per chain: (epoch, segments published)
+    uint32_t epoch;
+    float* ring;          // per chain: KH x [kN][kP] fp32, the state leaving a segment
+    unsigned int* status;
+    unsigned long long wait_limit;
+    uint32_t bar_counts[Smem::kNumBars];
+    int B, L;
+    int Ht;    // heads of kP channels (model heads x sub)
+    int Hr;    // model heads: dt [B][L][Hr], A and D [Hr]
+    int sub;   // kP-channel heads per model head
+    int G;
+    int N;     // state dim (<= kN)
+    int nkh;   // 64-wide halves of the state dim that hold data (1 or 2)
+    int gpr;   // head groups per batch row (Ht / KH)
+    int hpg;   // kP-channel heads per B/C group (Ht / G)
+    int ntiles, chains, seg_len, nseg, items;
+    int skip_publish;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __noinline__ void wait_gave_up(volatile int* abort_flag, unsigned int* status)
+{
+    record_status(status, kDevWaitTimeout);
+    *abort_flag = 1;
+}
+
+// Bounded wait of one thread that ignores the abort mode: true once the phase
+// completes, false after ~2 s (or kWaitPolls polls, whichever comes first).
+__device__ __forceinline__ bool wait_bounded_1(uint64_t* bar, uint32_t parity)
+{
+    if (mbar_try_wait_short(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait_short(bar, parity)) return true;
+        if ((it & 63u) == 0u && (it >= kWaitPolls || global_timer_ns() - t0 > kWaitNs)) return false;
+    }
+}
+
+// Bounded wait of one thread on an mbarrier phase (each poll may suspend the
+// thread for a short time, so a hand-off wakes the waiter promptly; the clock
+// is read every 64 polls). A give-up puts the CTA into abort mode: later waits
+// return at once and every role runs out its loop; the status word reports it.
+__device__ __forceinline__ void wait_bar_1(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                           unsigned int* status)
+{
+    if (*abort_flag) return;
+    if (mbar_try_wait_short(bar, parity)) return;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait_short(bar, parity)) return;
+        if ((it & 63u) == 0u && (it >= kWaitPolls || global_timer_ns() - t0 > kWaitNs)) break;
+    }
+    wait_gave_up(abort_flag, status);
+}
+
+// The same for a whole warp: lane 0 polls, and the warp leaves converged (the
+// tcgen05.ld / st / mma issue that follow a wait are .sync.aligned warp
+// instructions, which every lane must reach together; one poller also keeps
+// the barrier words' shared-memory traffic low).
+__device__ __forceinline__ void wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                         unsigned int* status)
+{
+    if ((threadIdx.x & 31) == 0) wait_bar_1(bar, parity, abort_flag, status);
+    __syncwarp();
+}
+
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity)
+{
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0) ok = wait_bounded_1(bar, parity) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// A segment of one chain: its batch row, head group and tiles.
+struct Pos {
+    int item, seg, chain, b, hs0, g, tile, tile_end;
+    bool valid;
+
+    __device__ __noinline__ void decode(const GParams& p, int it, int kh)
+    {
+        item = it;
+        valid = it >= 0 && it < p.items;
+        if (!valid) return;
+        seg = it / p.chains;
+        chain = it - seg * p.chains;
+        b = chain / p.gpr;
+        hs0 = (chain - b * p.gpr) * kh;
+        g = hs0 / p.hpg;
+        tile = seg * p.seg_len;
+        tile_end = min(tile + p.seg_len, p.ntiles);
+    }
+};
+
+// Ticket ring: the producer pushes segment numbers, warps 1..12 read each one.
+struct SchedReader {
+    uint32_t n = 0;
+    // Every reader sees the same sequence (the producer never overwrites an
+    // unread slot and pushes -1 to end it), so the warps of one role walk the
+    // same tiles. A reader that waits in vain (the producer is gone) ends its
+    // sequence after the bounded wait; in abort mode every reader ends at once
+    // (the roles are linked by mbarriers only, so no role waits on a warp
+    // that has left its loop for longer than a bounded wait).
+    __device__ int pop(uint8_t* sm, uint64_t* bars, volatile int* abort_flag, unsigned int* status)
+    {
+        if (*abort_flag) return -1;  // aborted: the results are undefined, every role just ends
+        const uint32_t slot = n % kSchedSlots;
+        const bool ok = wait_bounded(bars + kSchedFull + slot, (n / kSchedSlots) & 1);
+        const int it = ok ? *reinterpret_cast<volatile int*>(sm + Smem::kSched + slot * 4) : -1;
+        if (!ok && (threadIdx.x & 31) == 0) wait_gave_up(abort_flag, status);
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) mbar_arrive(bars + kSchedEmpty + slot);
+        ++n;
+        return it;
+    }
+};
+
+template <int KH>
+struct Walker {
+    Pos s;
+    SchedReader rd;
+    __device__ void begin(const GParams& p, uint8_t* sm, uint64_t* bars, volatile int* ab)
+    {
+        s.decode(p, rd.pop(sm, bars, ab, p.status), KH);
+    }
+    __device__ void next(const GParams& p, uint8_t* sm, uint64_t* bars, volatile int* ab)
+    {
+        if (++s.tile >= s.tile_end) s.decode(p, rd.pop(sm, bars, ab, p.status), KH);
+    }
+};
+
+template <int KH>
+__global__ void __launch_bounds__(kThreads, 1)
+grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
+                       const __grid_constant__ CUtensorMap tmB,
+                       const __grid_constant__ CUtensorMap tmC,
+                       const __grid_constant__ CUtensorMap tmY, const GParams p)
+{
+    extern __shared__ __align__(1024) uint8_t sm[];
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Smem::kBars);
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + Smem::kTmemPtr);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Smem::kAbort);
+    Rec* recs = reinterpret_cast<Rec*>(sm + Smem::kRec);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+
+    // the 128-byte swizzle needs 1024-byte aligned tiles; the layout above
+    // assumes the dynamic shared memory itself starts on such a boundary
+    if ((smem_addr(sm) & 1023u) != 0) {
+        if (tid == 0) record_status(p.status, kDevWaitTimeout);
+        return;
+    }
+    if (tid == 0) {
+        prefetch_tensormap(&tmX);
+        prefetch_tensormap(&tmB);
+        prefetch_tensormap(&tmC);
+        prefetch_tensormap(&tmY);
+        for (int i = 0; i < Smem::kNumBars; ++i) mbar_init(bars + i, p.bar_counts[i]);
+        mbar_fence_init();
+        *abort_flag = 0;
+    }
+    if (warp == kWarpProducer) {
+        tmem_alloc(s_tmem, kTmemCols);
+        tmem_relinquish();
+    }
+    if (p.nkh == 1) {
+        // N <= 64: the second halves of the C and B tiles are never loaded; zero
+        // them once so the states MMA (which spans all 128 state rows) reads zeros
+        for (int st = 0; st < 2; ++st)
+            for (int base = 0; base < 2; ++base) {
+                uint4* z = reinterpret_cast<uint4*>(sm + (base ? Smem::kB : Smem::kC) +
+                                                    st * 2 * kHalf + kHalf);
+                for (int u = tid; u < int(kHalf / 16); u += kThreads) z[u] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        fence_async_shared();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *s_tmem;
+
+    if (warp == kWarpProducer) {
+        // ------------------------------------------------------------ producer
+        // Tickets are taken one segment ahead, so that the L2 prefetch of the
+        // tiles kPrefetch ahead runs across segment boundaries too.
+        uint32_t npush = 0;
+        auto fetch = [&]() {
+            int it = -1;
+            if (lane == 0 && !*abort_flag) {
+                const unsigned int t = take_ticket(p.ctrl, p.epoch);
+                it = t < static_cast<unsigned int>(p.items) ? static_cast<int>(t) : -1;
+            }
+            return __shfl_sync(0xffffffffu, it, 0);
+        };
+        auto push = [&](int it) {
+            if (*abort_flag) return false;  // the readers end at once in abort mode
+            const uint32_t slot = npush % kSchedSlots;
+            // never overwrite a slot a reader has not taken yet, even when aborting
+            if (!wait_bounded(bars + kSchedEmpty + slot, ((npush / kSchedSlots) & 1) ^ 1)) {
+                if (lane == 0) wait_gave_up(abort_flag, p.status);
+                __syncwarp();
+                return false;
+            }
+            if (lane == 0) {
+                *reinterpret_cast<volatile int*>(sm + Smem::kSched + slot * 4) = it;
+                mbar_arrive(bars + kSchedFull + slot);
+            }
+            __syncwarp();
+            ++npush;
+            return true;
+        };
+        auto prefetch = [&](const Pos& q, int tile) {
+            const int t0 = tile * kT;
+            for (int h = 0; h < p.nkh; ++h) {
+                tma_prefetch_l2_4d(&tmC, h * 64, q.g, t0, q.b);
+                tma_prefetch_l2_4d(&tmB, h * 64, q.g, t0, q.b);
+            }
+#pragma unroll
+            for (int hh = 0; hh < KH; ++hh) tma_prefetch_l2_4d(&tmX, 0, q.hs0 + hh, t0, q.b);
+        };
+        Pos s, nx;
+        s.decode(p, fetch(), KH);
+        bool alive = push(s.valid ? s.item : -1);
+        nx.decode(p, s.valid ? fetch() : -1, KH);
+        int k = 0;
+        if (s.valid && elect_one_sync()) {
+            // the tiles before the prefetch distance
+            for (int d = 0; d < kPrefetch; ++d) {
+                if (s.tile + d < s.tile_end) prefetch(s, s.tile + d);
+                else if (nx.valid && nx.tile + (s.tile + d - s.tile_end) < nx.tile_end)
+                    prefetch(nx, nx.tile + (s.tile + d - s.tile_end));
+            }
+        }
+        __syncwarp();
+        while (alive && s.valid && !*abort_flag) {
+            const int st = k & 1;
+            const uint32_t par = ((k >> 1) & 1) ^ 1;
+            const int t0 = s.tile * kT;
+            // tile kPrefetch ahead into L2 (no shared memory, no completion)
+            if (kPrefetch > 0 && elect_one_sync()) {
+                const int ahead = s.tile + kPrefetch;
+                if (ahead < s.tile_end) prefetch(s, ahead);
+                else if (nx.valid && nx.tile + (ahead - s.tile_end) < nx.tile_end)
+                    prefetch(nx, nx.tile + (ahead - s.tile_end));
+            }
+            __syncwarp();
+            wait_bar(bars + kEmptyCB + st, par, abort_flag, p.status);
+            if (elect_one_sync()) {
+                mbar_arrive_expect_tx(bars + kFullCB + st, p.nkh * 2 * kHalf);
+                for (int q = 0; q < p.nkh; ++q) {
+                    tma_load_4d(sm + Smem::kC + st * 2 * kHalf + q * kHalf, &tmC, q * 64, s.g, t0, s.b,
+                                bars + kFullCB + st);
+                    tma_load_4d(sm + Smem::kB + st * 2 * kHalf + q * kHalf, &tmB, q * 64, s.g, t0, s.b,
+                                bars + kFullCB + st);
+                }
+            }
+            __syncwarp();
+            wait_bar(bars + kEmptyX + st, par, abort_flag, p.status);
+            if (elect_one_sync()) {
+                mbar_arrive_expect_tx(bars + kFullX + st, KH * kHalf);
+#pragma unroll
+                for (int hh = 0; hh < KH; ++hh)
+                    tma_load_4d(sm + Smem::kX + st * 2 * kHalf + hh * kHalf, &tmX, 0, s.hs0 + hh, t0, s.b,
+                                bars + kFullX + st);
+            }
+            __syncwarp();
+            ++k;
+            if (++s.tile >= s.tile_end) {
+                s = nx;
+                alive = push(s.valid ? s.item : -1);
+                nx.decode(p, s.valid ? fetch() : -1, KH);
+            }
+        }
+        if (alive && s.valid) push(-1);  // aborted: tell every role to stop
+        // every load issued has landed before the CTA can exit
+        for (int j = max(0, k - 2); j < k; ++j) {
+            wait_bounded(bars + kFullCB + (j & 1), (j >> 1) & 1);
+            wait_bounded(bars + kFullX + (j & 1), (j >> 1) & 1);
+        }
+    } else if (warp == kWarpMmaA) {
+        // ------------------------------------------------- stream A: MMA1, states
+        constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
+        constexpr uint32_t id_st = idesc_bf16(128, 64 * KH, true, true);
+        const uint64_t dc0 = sdesc_sw128(smem_addr(sm + Smem::kC), 16, 1024);
+        const uint64_t db0 = sdesc_sw128(smem_addr(sm + Smem::kB), 16, 1024);
+        const uint64_t dbt0 = sdesc_sw128(smem_addr(sm + Smem::kB), kHalf, 1024);  // B^T, MN-major
+        const uint64_t dx0 = sdesc_sw128(smem_addr(sm + Smem::kX), kHalf, 1024);   // X', MN-major
+        Walker<KH> w;
+        w.begin(p, sm, bars, abort_flag);
+        for (int k = 0; w.s.valid; ++k, w.next(p, sm, bars, abort_flag)) {
+            const int st = k & 1;
+            const uint32_t par = (k >> 1) & 1;
+            const uint64_t stage = static_cast<uint64_t>(st * 2 * kHalf) >> 4;
+            wait_bar(bars + kFullCB + st, par, abort_flag, p.status);
+            wait_bar(bars + kSFree + st, par ^ 1, abort_flag, p.status);  // MMA2 of tile k - 2
+            tc_fence_after_sync();
+            if (elect_one_sync()) {
+                for (int q = 0; q < 4 * p.nkh; ++q) {
+                    const uint32_t off = ((q >> 2) * kHalf + (q & 3) * 32) >> 4;
+                    mma_bf16(tmem + kColS + st * 128, dc0 + stage + off, db0 + stage + off, id_s, q > 0);
+                }
+                mma_commit(bars + kSFull + st);
+            }
+            __syncwarp();
+            wait_bar(bars + kXpFull + st, par, abort_flag, p.status);
+            wait_bar(bars + kHReady, k & 1, abort_flag, p.status);
+            tc_fence_after_sync();
+            if (elect_one_sync()) {
+#pragma unroll
+                for (int q = 0; q < kT / 16; ++q)
+                    mma_bf16(tmem + kColH, dbt0 + stage + q * (2048 >> 4), dx0 + stage + q * (2048 >> 4),
+                             id_st, true);
+                mma_commit(bars + kStatesDone);
+                mma_commit(bars + kXRead + st);
+                mma_commit(bars + kEmptyCB + st);
+                mma_commit(bars + kEmptyX + st);
+            }
+            __syncwarp();
+        }
+        if (elect_one_sync()) mma_commit(bars + kDrainA);
+        __syncwarp();
+        wait_bounded(bars + kDrainA, 0);
+    } else if (warp == kWarpMmaB) {
+        // -------------------------------------------------- stream B: MMA3, MMA2
+        constexpr uint32_t id_y = idesc_bf16(128, 64 * KH, false, true);
+        constexpr uint32_t id_y1 = idesc_bf16(128, 64, false, true);
+        const uint64_t dc0 = sdesc_sw128(smem_addr(sm + Smem::kC), 16, 1024);
+        const uint64_t dhp = sdesc_sw128(smem_addr(sm + Smem::kHp), kHalf, 1024);
+        const uint64_t dx0 = sdesc_sw128(smem_addr(sm + Smem::kX), kHalf, 1024);
+        Walker<KH> w;
+        w.begin(p, sm, bars, abort_flag);
+        uint32_t nh = 0;  // exact-form tiles so far
+        for (int k = 0; w.s.valid; ++k, w.next(p, sm, bars, abort_flag)) {
+            const int st = k & 1;
+            const uint32_t par = (k >> 1) & 1;
+            const uint64_t stage = static_cast<uint64_t>(st * 2 * kHalf) >> 4;
+            wait_bar(bars + kRecFull + st, par, abort_flag, p.status);
+            const bool hard = recs[st].hard != 0;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars + kRecEmpty + st);
+            wait_bar(bars + kFullCB + st, par, abort_flag, p.status);
+            wait_bar(bars + kHpFull, k & 1, abort_flag, p.status);
+            wait_bar(bars + kZEmpty, (k & 1) ^ 1, abort_flag, p.status);
+            tc_fence_after_sync();
+            if (elect_one_sync()) {
+                for (int q = 0; q < 4 * p.nkh; ++q)
+                    mma_bf16(tmem + kColZ, dc0 + stage + (((q >> 2) * kHalf + (q & 3) * 32) >> 4),
+                             dhp + q * (2048 >> 4), id_y, q > 0);
+            }
+            __syncwarp();
+            if (!hard) {
+                if (elect_one_sync()) {
+                    mma_commit(bars + kHpEmpty);
+                    mma_commit(bars + kEmptyCB + st);
+                }
+                __syncwarp();
+                wait_bar(bars + kTrilFull + st, par, abort_flag, p.status);
+                wait_bar(bars + kXpFull + st, par, abort_flag, p.status);
+                tc_fence_after_sync();
+                if (elect_one_sync()) {
+#pragma unroll
+                    for (int q = 0; q < kT / 16; ++q)
+                        mma_bf16_tmem_a(tmem + kColZ, tmem + kColS + st * 128 + q * 8,
+                                        dx0 + stage + q * (2048 >> 4), id_y, true);
+                    mma_commit(bars + kZFull);
+                    mma_commit(bars + kEmptyX + st);
+                    mma_commit(bars + kSFree + st);
+                }
+                __syncwarp();
+            } else {
+                // exact form: raw X into the H' buffer once MMA3 has read it,
+                // Z scaled by the output warps, then one masked product per head
+                if (elect_one_sync()) {
+                    mma_commit(bars + kEmptyCB + st);
+                    mma_commit(bars + kM3Done);
+                }
+                __syncwarp();
+                wait_bar(bars + kM3Done, nh & 1, abort_flag, p.status);
+                if (elect_one_sync()) {
+                    mbar_arrive_expect_tx(bars + kRawX, KH * kHalf);
+#pragma unroll
+                    for (int hh = 0; hh < KH; ++hh)
+                        tma_load_4d(sm + Smem::kHp + hh * kHalf, &tmX, 0, w.s.hs0 + hh, w.s.tile * kT, w.s.b,
+                                    bars + kRawX);
+                }
+                __syncwarp();
+                wait_bar(bars + kRawX, nh & 1, abort_flag, p.status);
+                wait_bar(bars + kZScaled, nh & 1, abort_flag, p.status);
+#pragma unroll
+                for (int hh = 0; hh < KH; ++hh) {
+                    const uint32_t u = nh * KH + hh;
+                    wait_bar(bars + kSlotFull, u & 1, abort_flag, p.status);
+                    tc_fence_after_sync();
+                    if (elect_one_sync()) {
+#pragma unroll
+                        for (int q = 0; q < kT / 16; ++q)
+                            mma_bf16_tmem_a(tmem + kColZ + hh * 64, tmem + kColS + st * 128 + 64 + q * 8,
+                                            dhp + ((hh * kHalf) >> 4) + q * (2048 >> 4), id_y1, true);
+                        mma_commit(bars + kSlotFree);
+                    }
+                    __syncwarp();
+                }
+                if (elect_one_sync()) {
+                    mma_commit(bars + kZFull);
+                    mma_commit(bars + kEmptyX + st);
+                    mma_commit(bars + kSFree + st);
+                    mma_commit(bars + kHpEmpty);
+                }
+                __syncwarp();
+                ++nh;
+            }
+        }
+        if (elect_one_sync()) mma_commit(bars + kDrainB);
+        __syncwarp();
+        wait_bounded(bars + kDrainB, 0);
+    } else if (warp == kWarpPro0 || warp == kWarpPro1) {
+        // ---------------------------------------- prologue: decay, record (one head)
+        const int hh = warp == kWarpPro0 ? 0 : 1;
+        Walker<KH> w;
+        w.begin(p, sm, bars, abort_flag);
+        if (hh < KH) {
+            // lane l holds tokens l, l + 32, l + 64, l + 96 of the tile
+            float dtv[4];
+            float Aval = 0.f;
+            auto fetch = [&](const Pos& q) {
+                const int rows = min(kT, p.L - q.tile * kT);
+                const int hr = (q.hs0 + hh) / p.sub;
+                const size_t base = (static_cast<size_t>(q.b) * p.L + q.tile * kT) * p.Hr + hr;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int j = lane + 32 * u;
+                    dtv[u] = j < rows ? __ldg(p.dt + base + static_cast<size_t>(j) * p.Hr) : 0.f;
+                }
+                Aval = __ldg(p.A + hr);
+            };
+            if (w.s.valid) fetch(w.s);
+            for (int k = 0; w.s.valid; ++k) {
+                const int st = k & 1;
+                const uint32_t par = (k >> 1) & 1;
+                const float dtc[4] = {dtv[0], dtv[1], dtv[2], dtv[3]};
+                const float Ah = Aval * kLog2e;
+                w.next(p, sm, bars, abort_flag);
+                if (w.s.valid) fetch(w.s);  // next tile's dt, in flight during this one
+
+                Rec& r = recs[st];
+                wait_bar(bars + kRecEmpty + st, par ^ 1, abort_flag, p.status);
+                float cs[4];
+                float carry = 0.f;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    float v = dtc[u] * Ah;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const float t = __shfl_up_sync(0xffffffffu, v, o);
+                        if (lane >= o) v += t;
+                    }
+                    cs[u] = v + carry;
+                    carry += __shfl_sync(0xffffffffu, v, 31);
+                }
+                const float cs_end = carry;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) r.cs[hh][lane + 32 * u] = cs[u];
+                const int hard_h = -cs_end > kHardLog2 ? 1 : 0;
+                int hard = hard_h;
+                if (KH == 2) {
+                    if (lane == 0) {
+                        r.hardh[hh] = hard_h;
+                        mbar_arrive(bars + kHx);
+                    }
+                    wait_bar(bars + kHx, k & 1, abort_flag, p.status);
+                    hard = r.hardh[0] | r.hardh[1];
+                }
+                const float cref = 0.5f * cs_end;
+                if (lane == 0) {
+                    r.cref[hh] = cref;
+                    r.csend[hh] = cs_end;
+                    r.hard = hard;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bars + kRecFull + st);
+            }
+        } else {
+            while (w.s.valid) w.next(p, sm, bars, abort_flag);  // KH = 1: read the tickets only
+        }
+    } else if (warp >= kWgState && warp < kWgState + 4) {
+        // ------------- state: H', the scaled h, segment hand-off; mask: tril(S)
+        const int wq = warp - kWgState;
+        const int r = wq * 32 + lane;  // state row n, token row i = TMEM lane
+        const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+        const size_t Nst = static_cast<size_t>(p.N);
+        const bool n_live = r < p.N;  // state rows past N are zero padding
+        Walker<KH> w;
+        w.begin(p, sm, bars, abort_flag);
+        float s_pend[KH];  // true h = s_pend * (h in TMEM)
+#pragma unroll
+        for (int hh = 0; hh < KH; ++hh) s_pend[hh] = 1.f;
+        Pos prev;
+        prev.valid = false;
+        bool prev_last = false;
+        uint32_t npub = 0;  // segment end states published so far
+        uint32_t nh = 0;    // exact-form tiles so far
+
+        for (int k = 0;; ++k) {
+            const bool have = w.s.valid;
+            // ---- the state after tile k - 1: hand it off if its segment ends there
+            if (k >= 1) {
+                wait_bar(bars + kStatesDone, (k - 1) & 1, abort_flag, p.status);
+                tc_fence_after_sync();
+                if (prev_last) {
+                    const bool fin = prev.tile == p.ntiles - 1;
+#pragma unroll
+                    for (int hh = 0; hh < KH; ++hh) {
+#pragma unroll 1
+                        for (int half = 0; half < 2; ++half) {
+                            float v[32];
+                            tmem_ld32(tmem + lane_off + kColH + hh * 64 + half * 32, v);
+                            tmem_wait_ld();
+                            if (fin) {
+                                if (p.final_state && n_live) {
+                                    float* dst = p.final_state +
+                                                 ((static_cast<size_t>(prev.b) * p.Ht + prev.hs0 + hh) * kP +
+                                                  half * 32) * Nst + r;
+#pragma unroll
+                                    for (int q = 0; q < 32; ++q) dst[q * Nst] = s_pend[hh] * v[q];
+                                }
+                            } else {
+                                float4* dst = reinterpret_cast<float4*>(
+                                    p.ring + ((static_cast<size_t>(prev.chain) * KH + hh) * kN + r) * kP +
+                                    half * 32);
+#pragma unroll
+                                for (int q = 0; q < 8; ++q)
+                                    dst[q] = make_float4(s_pend[hh] * v[4 * q], s_pend[hh] * v[4 * q + 1],
+                                                         s_pend[hh] * v[4 * q + 2], s_pend[hh] * v[4 * q + 3]);
+                            }
+                        }
+                    }
+                    if (!fin) {
+                        // every thread's part is visible GPU-wide before the four
+                        // warps report to thread 0, which then releases the flag
+                        __threadfence();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bars + kPub);
+                        if (r == 0) {
+                            wait_bar_1(bars + kPub, npub & 1, abort_flag, p.status);
+                            __threadfence();
+                            if (!p.skip_publish)
+                                st_release_gpu_u64(p.flags + prev.chain,
+                                                   tagged(p.epoch, static_cast<uint32_t>(prev.seg + 1)));
+                        }
+                        __syncwarp();
+                        ++npub;
+                    }
+                }
+            }
+            if (!have) break;
+            // ---- the record of tile k (released after the mask)
+            const int st = k & 1;
+            const uint32_t par = (k >> 1) & 1;
+            const Rec& rc = recs[st];
+            float sig3[KH], sigst[KH], snext[KH];
+            wait_bar(bars + kRecFull + st, par, abort_flag, p.status);
+            const bool hard = rc.hard != 0;
+#pragma unroll
+            for (int hh = 0; hh < KH; ++hh) {
+                const float c = rc.cref[hh], ce = rc.csend[hh];
+                sig3[hh] = hard ? 1.f : ex2_approx(c);
+                sigst[hh] = ex2_approx(hard ? ce : c);
+                snext[hh] = hard ? 1.f : ex2_approx(ce - c);
+            }
+            // ---- H' (bf16 operand of MMA3) and the scaled state for tile k
+            const bool first = w.s.tile == w.s.seg * p.seg_len;
+            if (first && w.s.seg > 0) {
+                // bounded acquire poll on the predecessor's flag, one per warp.
+                // Giving up only records the status: the call's results are
+                // then undefined, but every role still runs to its end.
+                if (lane == 0 && !*abort_flag) {
+                    const unsigned long long* f = p.flags + w.s.chain;
+                    bool ok = false;
+                    const uint64_t t0 = global_timer_ns();
+                    for (unsigned long long it = 0; it < p.wait_limit; ++it) {
+                        const uint64_t v = ld_acquire_gpu_u64(f);
+                        if (static_cast<uint32_t>(v >> 32) == p.epoch &&
+                            static_cast<uint32_t>(v) >= static_cast<uint32_t>(w.s.seg)) {
+                            ok = true;
+                            break;
+                        }
+                        if ((it & 255) == 255 && global_timer_ns() - t0 > 4000000000ull) break;
+                        __nanosleep(64);
+                    }
+                    if (!ok) record_status(p.status, kDevWaitTimeout);
+                }
+                __syncwarp();
+            }
+            wait_bar(bars + kHpEmpty, (k & 1) ^ 1, abort_flag, p.status);
+            tc_fence_after_sync();
+#pragma unroll
+            for (int hh = 0; hh < KH; ++hh) {
+                if (first) s_pend[hh] = 1.f;
+                const float f3 = sig3[hh] * s_pend[hh], fst = sigst[hh] * s_pend[hh];
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    float v[32];
+                    const uint32_t a = tmem + lane_off + kColH + hh * 64 + half * 32;
+                    if (!first) {
+                        tmem_ld32(a, v);
+                        tmem_wait_ld();
+                    } else if (w.s.seg > 0) {
+                        // what the predecessor published: row r of [kN][kP]
+                        const float4* src = reinterpret_cast<const float4*>(
+                            p.ring + ((static_cast<size_t>(w.s.chain) * KH + hh) * kN + r) * kP + half * 32);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 u = __ldcg(src + q);
+                            v[4 * q] = u.x;
+                            v[4 * q + 1] = u.y;
+                            v[4 * q + 2] = u.z;
+                            v[4 * q + 3] = u.w;
+                        }
+                    } else if (p.init && n_live) {
+                        // the chain's initial state, [B][H][P][N]
+                        const float* src = p.init +
+                                           ((static_cast<size_t>(w.s.b) * p.Ht + w.s.hs0 + hh) * kP + half * 32) *
+                                               Nst + r;
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) v[q] = __ldg(src + q * Nst);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) v[q] = 0.f;
+                    }
+                    uint8_t* row = sm + Smem::kHp + hh * kHalf + r * 128;
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) {
+                        const int chunk = half * 4 + cc;
+                        const uint4 hv = make_uint4(pack_bf16x2(f3 * v[cc * 8 + 0], f3 * v[cc * 8 + 1]),
+                                                    pack_bf16x2(f3 * v[cc * 8 + 2], f3 * v[cc * 8 + 3]),
+                                                    pack_bf16x2(f3 * v[cc * 8 + 4], f3 * v[cc * 8 + 5]),
+                                                    pack_bf16x2(f3 * v[cc * 8 + 6], f3 * v[cc * 8 + 7]));
+                        *reinterpret_cast<uint4*>(row + (((chunk ^ r) & 7) << 4)) = hv;
+                    }
+                    uint32_t o[32];
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(fst * v[q]);
+                    tmem_st32(a, o);
+                }
+                s_pend[hh] = snext[hh];
+            }
+            tmem_wait_st();
+            fence_async_shared();
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bars + kHReady);
+                mbar_arrive(bars + kHpFull);
+            }
+
+            // ---- mask of tile k: S -> tril(S), as bf16 pairs over the first 64
+            // columns of the S buffer (block jb of 32 fp32 columns lands on
+            // columns 16 jb .. 16 jb + 15, which are already read)
+            wait_bar(bars + kSFull + st, par, abort_flag, p.status);
+            tc_fence_after_sync();
+            const uint32_t s_col = tmem + lane_off + kColS + st * 128;
+#pragma unroll 1
+            for (int jb = 0; jb < 4; ++jb) {
+                uint32_t packed[16];
+                if (jb <= wq) {
+                    float sv[32];
+                    tmem_ld32(s_col + jb * 32, sv);
+                    tmem_wait_ld();
+                    if (jb == wq) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) sv[e] = e <= lane ? sv[e] : 0.f;
+                    }
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) packed[q] = pack_bf16x2(sv[2 * q], sv[2 * q + 1]);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) packed[q] = 0u;
+                }
+                tmem_st16(s_col + jb * 16, packed);
+            }
+            tmem_wait_st();
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars + kTrilFull + st);
+            if (hard) {
+                // exact form: S~_h,ij = tril(S)_ij 2^(cs_i - cs_j) dt_j into
+                // columns 64-127, one head at a time
+                const int rows = min(kT, p.L - w.s.tile * kT);
+#pragma unroll
+                for (int hh = 0; hh < KH; ++hh) {
+                    const int hr = (w.s.hs0 + hh) / p.sub;
+                    const size_t base = (static_cast<size_t>(w.s.b) * p.L + w.s.tile * kT) * p.Hr + hr;
+                    float dtl[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int j = lane + 32 * u;
+                        dtl[u] = j < rows ? __ldg(p.dt + base + static_cast<size_t>(j) * p.Hr) : 0.f;
+                    }
+                    const float cs_i = rc.cs[hh][r];
+                    const uint32_t u_slot = nh * KH + hh;
+                    wait_bar(bars + kSlotFree, (u_slot & 1) ^ 1, abort_flag, p.status);
+                    tc_fence_after_sync();
+#pragma unroll 1
+                    for (int half = 0; half < 2; ++half) {
+                        uint32_t wv[32];
+                        float tv[32];
+                        tmem_ld32(s_col + half * 32, tv);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) wv[e] = __float_as_uint(tv[e]);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int j0 = half * 64 + 2 * e;  // tokens j0, j0 + 1 (same 32-block)
+                            const float dsrc = half ? dtl[2 + (e >> 4)] : dtl[e >> 4];
+                            const float d0 = __shfl_sync(0xffffffffu, dsrc, j0 & 31);
+                            const float d1 = __shfl_sync(0xffffffffu, dsrc, (j0 + 1) & 31);
+                            const float m0 = ex2_approx(fminf(cs_i - rc.cs[hh][j0], 0.f)) * d0;
+                            const float m1 = ex2_approx(fminf(cs_i - rc.cs[hh][j0 + 1], 0.f)) * d1;
+                            wv[e] = pack_bf16x2(bf16_lo(wv[e]) * m0, bf16_hi(wv[e]) * m1);
+                        }
+                        tmem_st32(s_col + 64 + half * 32, wv);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bars + kSlotFull);
+                }
+                ++nh;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars + kRecEmpty + st);
+            prev = w.s;
+            prev_last = w.s.tile == w.s.tile_end - 1;
+            w.next(p, sm, bars, abort_flag);
+        }
+    } else if (warp >= kWgOut && warp < kWgOut + 4) {
+        // -------------------------- output: X' in place, then y = e Z + D x.
+        // Thread r owns token row r of a tile: it writes X'_r = f_r x_r over
+        // the row of x, and later y_r over X'_r, taking x_r for the D term back
+        // as X'_r / f_r (one more bf16 rounding of that term), or from global
+        // memory where f_r is too small for that (dt_r = 0, or an early token
+        // of an exact-form tile); one TMA store per head then writes the tile
+        // (rows past L are clipped). X' of tile k + 1 is built before the
+        // output of tile k, so that its products are not held up by the
+        // output. Exact form: first Z_r *= 2^(cs_r), which the per-head
+        // masked products then add to.
+        const int wq = warp - kWgOut;
+        const int r = wq * 32 + lane;  // token row i = TMEM lane
+        const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+        struct TileOut {
+            Pos pos;
+            float f[KH], e[KH], zs[KH], Dh[KH];
+            bool hard;
+        };
+        Walker<KH> w;
+        w.begin(p, sm, bars, abort_flag);
+        TileOut cur, nxt;
+        bool have_cur = false;
+        uint32_t nh = 0;
+        int k = 0;  // the tile whose output is pending; X' is built for tile k + have_cur
+        for (;;) {
+            const bool have_nx = w.s.valid;
+            if (have_nx) {
+                // ---- X' of the next tile
+                const int kx = k + (have_cur ? 1 : 0);
+                const int st = kx & 1;
+                const uint32_t par = (kx >> 1) & 1;
+                nxt.pos = w.s;
+                const bool live = r < p.L - w.s.tile * kT;
+                float dtr[KH];
+#pragma unroll
+                for (int hh = 0; hh < KH; ++hh) {
+                    const int hr = (w.s.hs0 + hh) / p.sub;
+                    dtr[hh] = live ? __ldg(p.dt + (static_cast<size_t>(w.s.b) * p.L + w.s.tile * kT + r) * p.Hr + hr)
+                                   : 0.f;
+                    nxt.Dh[hh] = p.D ? __ldg(p.D + hr) : 0.f;
+                }
+                const Rec& rc = recs[st];
+                wait_bar(bars + kRecFull + st, par, abort_flag, p.status);
+                nxt.hard = rc.hard != 0;
+#pragma unroll
+                for (int hh = 0; hh < KH; ++hh) {
+                    const float ci = rc.cs[hh][r];
+                    nxt.f[hh] = ex2_approx(nxt.hard ? rc.csend[hh] - ci : rc.cref[hh] - ci) * dtr[hh];
+                    nxt.e[hh] = nxt.hard ? 1.f : ex2_approx(ci - rc.cref[hh]);
+                    nxt.zs[hh] = ex2_approx(ci);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bars + kRecEmpty + st);
+                // X' = diag(f) X in place, in fp32 with one rounding
+                wait_bar(bars + kFullX + st, par, abort_flag, p.status);
+                uint8_t* xs = sm + Smem::kX + st * 2 * kHalf;
+#pragma unroll
+                for (int hh = 0; hh < KH; ++hh) {
+                    uint8_t* row = xs + hh * kHalf + r * 128;
+                    const float fh = nxt.f[hh];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        uint4* a = reinterpret_cast<uint4*>(row + (((c ^ r) & 7) << 4));
+                        const uint4 v = *a;
+                        *a = make_uint4(pack_bf16x2(fh * bf16_lo(v.x), fh * bf16_hi(v.x)),
+                                        pack_bf16x2(fh * bf16_lo(v.y), fh * bf16_hi(v.y)),
+                                        pack_bf16x2(fh * bf16_lo(v.z), fh * bf16_hi(v.z)),
+                                        pack_bf16x2(fh * bf16_lo(v.w), fh * bf16_hi(v.w)));
+                    }
+                }
+                fence_async_shared();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bars + kXpFull + st);
+            }
+            if (have_cur) {
+                // ---- output of tile k
+                const int st = k & 1;
+                uint8_t* xs = sm + Smem::kX + st * 2 * kHalf;
+                if (cur.hard) {
+                    wait_bar(bars + kM3Done, nh & 1, abort_flag, p.status);
+                    tc_fence_after_sync();
+#pragma unroll
+                    for (int hh = 0; hh < KH; ++hh) {
+#pragma unroll 1
+                        for (int qd = 0; qd < 4; ++qd) {
+                            float v[16];
+                            uint32_t o[16];
+                            const uint32_t a = tmem + lane_off + kColZ + hh * 64 + qd * 16;
+                            tmem_ld16(a, v);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int q = 0; q < 16; ++q) o[q] = __float_as_uint(v[q] * cur.zs[hh]);
+                            tmem_st16(a, o);
+                        }
+                    }
+                    tmem_wait_st();
+                    tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bars + kZScaled);
+                    ++nh;
+                }
+                // y over X' once MMA2 (Z full) and the states MMA have read it.
+                // (A per-stage barrier: the single-phase "states done" could
+                // already have completed for tile k + 1, whose X' is built above.)
+                wait_bar(bars + kZFull, k & 1, abort_flag, p.status);
+                wait_bar(bars + kXRead + st, (k >> 1) & 1, abort_flag, p.status);
+                tc_fence_after_sync();
+                const bool live = r < p.L - cur.pos.tile * kT;
+#pragma unroll
+                for (int hh = 0; hh < KH; ++hh) {
+                    uint8_t* row = xs + hh * kHalf + r * 128;
+                    // D x_r from X'_r / f_r, or from global memory where f_r is tiny
+                    const bool from_xp = cur.f[hh] >= 0x1p-100f;
+                    const float dx = from_xp ? cur.Dh[hh] / cur.f[hh] : cur.Dh[hh];
+                    const uint4* xg = reinterpret_cast<const uint4*>(
+                        p.x + ((static_cast<size_t>(cur.pos.b) * p.L + cur.pos.tile * kT + r) * p.Ht +
+                               cur.pos.hs0 + hh) * kP);
+#pragma unroll
+                    for (int qd = 0; qd < 4; ++qd) {
+                        float zv[16];
+                        tmem_ld16(tmem + lane_off + kColZ + hh * 64 + qd * 16, zv);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int q = 0; q < 2; ++q) {
+                            const int c = qd * 2 + q;
+                            uint4* a = reinterpret_cast<uint4*>(row + (((c ^ r) & 7) << 4));
+                            uint4 xq = *a;
+                            if (!from_xp)
+                                xq = (live && cur.Dh[hh] != 0.f) ? __ldg(xg + c) : make_uint4(0u, 0u, 0u, 0u);
+                            const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
+                            uint32_t o[4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const int j = q * 8 + u * 2;
+                                o[u] = pack_bf16x2(fmaf(cur.e[hh], zv[j], dx * bf16_lo(xw[u])),
+                                                   fmaf(cur.e[hh], zv[j + 1], dx * bf16_hi(xw[u])));
+                            }
+                            *a = make_uint4(o[0], o[1], o[2], o[3]);
+                        }
+                    }
+                }
+                tc_fence_before_sync();
+                fence_async_shared();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(bars + kZEmpty);
+                    mbar_arrive(bars + kYStaged);
+                }
+                if (r == 0) {
+                    // one TMA store per head once all four warps staged their rows;
+                    // the stage returns to the producer when the stores have read it
+                    wait_bar_1(bars + kYStaged, k & 1, abort_flag, p.status);
+#pragma unroll
+                    for (int hh = 0; hh < KH; ++hh)
+                        tma_store_4d(&tmY, xs + hh * kHalf, 0, cur.pos.hs0 + hh, cur.pos.tile * kT, cur.pos.b);
+                    tma_store_commit();
+                    tma_store_wait_read();
+                    mbar_arrive(bars + kEmptyX + st);
+                }
+                __syncwarp();
+                ++k;
+            }
+            if (!have_nx) break;
+            cur = nxt;
+            have_cur = true;
+            w.next(p, sm, bars, abort_flag);
+        }
+        if (r == 0) tma_store_wait_all();
+    }
+
+    // ---- teardown
+    __syncwarp();
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == kWarpProducer) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ------------------------------------------------------------------ host side
+
+int heads_per_tile(const FwdArgs& a)
+{
+    const int Ht = a.H * (a.P / kP);
+    return (Ht / a.G) % 2 == 0 ? 2 : 1;
+}
+
+struct Plan {
+    int KH, Ht, chains, ntiles, seg_len, nseg, items, grid;
+    size_t ws_ctrl, ws_flags, ws_ring, ws_total;
+};
+
+// Segments per chain: about `per_cta` segments per CTA in all.
+constexpr int kItemsPerCta = 4;
+
+Plan make_plan(const FwdArgs& a, int ctas)
+{
+    Plan g;
+    g.KH = heads_per_tile(a);
+    g.Ht = a.H * (a.P / kP);
+    g.chains = a.B * (g.Ht / g.KH);
+    g.ntiles = (a.L + kT - 1) / kT;
+    long long want = (static_cast<long long>(kItemsPerCta) * ctas + g.chains - 1) / g.chains;
+    if (want < 1) want = 1;
+    if (want > g.ntiles) want = g.ntiles;
+    g.seg_len = static_cast<int>((g.ntiles + want - 1) / want);
+    g.nseg = (g.ntiles + g.seg_len - 1) / g.seg_len;
+    g.items = g.chains * g.nseg;
+    g.grid = g.items < ctas ? g.items : ctas;
+    g.ws_ctrl = 0;
+    g.ws_flags = 256;
+    g.ws_ring = g.ws_flags + ((static_cast<size_t>(g.chains) * 8 + 255) / 256) * 256;
+    g.ws_total = g.ws_ring + static_cast<size_t>(g.chains) * g.KH * kN * kP * sizeof(float);
+    return g;
+}
+
+int g_skip_publish = 0;
+
+template <int KH>
+cudaError_t launch_kh(const CUtensorMap& tmX, const CUtensorMap& tmB, const CUtensorMap& tmC,
+                      const CUtensorMap& tmY, const GParams& p, int grid, cudaStream_t stream)
+{
+    const uint32_t smem = Smem::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(grouped_forward_kernel<KH>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    grouped_forward_kernel<KH><<<grid, kThreads, smem, stream>>>(tmX, tmB, tmC, tmY, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool supported(const FwdArgs& a)
+{
+    return a.bf16 && a.P % kP == 0 && a.P >= kP && a.N % 8 == 0 && a.N >= 8 && a.N <= kN &&
+           (a.chunk == 64 || a.chunk == 128 || a.chunk == 256) &&
+           static_cast<long long>(a.B) * a.L > 0;
+}
+
+bool preferred(const FwdArgs& a, int ctas)
+{
+    if (!supported(a)) return false;
+    const Plan g = make_plan(a, ctas);
+    // segments of one chain wait on each other in turn; with fewer chains than
+    // CTAs they would run one after another, which the segment-parallel form
+    // of the per-head kernel avoids
+    return g.chains >= ctas / 2 || g.nseg == 1;
+}
+
+size_t workspace_bytes(const FwdArgs& a, int ctas) { return make_plan(a, ctas).ws_total; }
+
+void set_skip_publish(int v) { g_skip_publish = v; }
+
+cudaError_t forward(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)
+{
+    if (!supported(a)) return cudaErrorInvalidValue;
+    const int ctas = ctx.num_sms > 0 ? ctx.num_sms : 1;
+    const Plan g = make_plan(a, ctas);
+    CUtensorMap tmX, tmB, tmC, tmY;
+    if (!make_map_bf16_4d(&tmX, a.x, kP, g.Ht, a.L, a.B) ||
+        !make_map_bf16_4d(&tmY, a.y, kP, g.Ht, a.L, a.B) ||
+        !make_map_bf16_4d(&tmB, a.Bm, a.N, a.G, a.L, a.B) ||
+        !make_map_bf16_4d(&tmC, a.Cm, a.N, a.G, a.L, a.B))
+        return cudaErrorInvalidValue;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    GParams p;
+    p.dt = a.dt;
+    p.A = a.A;
+    p.D = a.D;
+    p.init = a.init;
+    p.x = static_cast<const __nv_bfloat16*>(a.x);
+    p.y = static_cast<__nv_bfloat16*>(a.y);
+    p.final_state = a.final_state;
+    p.ctrl = reinterpret_cast<unsigned long long*>(ws + g.ws_ctrl);
+    p.flags = reinterpret_cast<unsigned long long*>(ws + g.ws_flags);
+    p.epoch = ctx.epoch;
+    p.ring = reinterpret_cast<float*>(ws + g.ws_ring);
+    p.status = ctx.status;
+    p.wait_limit = ctx.wait_limit;
+    for (int i = 0; i < Smem::kNumBars; ++i) p.bar_counts[i] = bar_count(i, g.KH);
+    p.B = a.B;
+    p.L = a.L;
+    p.Ht = g.Ht;
+    p.Hr = a.H;
+    p.sub = a.P / kP;
+    p.G = a.G;
+    p.N = a.N;
+    p.nkh = a.N <= 64 ? 1 : 2;
+    p.gpr = g.Ht / g.KH;
+    p.hpg = g.Ht / a.G;
+    p.ntiles = g.ntiles;
+    p.chains = g.chains;
+    p.seg_len = g.seg_len;
+    p.nseg = g.nseg;
+    p.items = g.items;
+    p.skip_publish = g_skip_publish;
+    return g.KH == 2 ? launch_kh<2>(tmX, tmB, tmC, tmY, p, g.grid, ctx.stream)
+                     : launch_kh<1>(tmX, tmB, tmC, tmY, p, g.grid, ctx.stream);
+}
+
+}  // namespace grouped
+}  // namespace ssd

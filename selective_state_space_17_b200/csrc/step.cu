@@ -9,15 +9,16 @@
 // The step is bound by HBM: the fp32 state is read and written once (P*N*8
 // bytes per head) and everything else is small. One CTA of 8 warps per (b, h);
 // a warp owns whole state rows p and moves them with 128-bit accesses (lane l
-// holds n = 4l .. 4l+3 of each 128-column stripe), four rows in flight per
-// warp, and reduces y_p with shuffles.
+// holds n = 4l .. 4l+3 of each 128-column stripe), eight rows in flight per
+// warp (a whole 64 x 128 head's state per CTA, so that enough bytes are in
+// flight to cover the HBM latency), and reduces y_p with shuffles.
 #include "common.cuh"
 
 namespace ssd {
 namespace {
 
 constexpr int kWarps = 8;
-constexpr int kRowsInFlight = 4;
+constexpr int kRowsInFlight = 8;
 
 template <typename T>
 __device__ __forceinline__ float4 load4(const T* p);
@@ -47,7 +48,7 @@ __device__ __forceinline__ float warp_sum(float v)
 
 // Vector path: N % 4 == 0 (every row starts 16-byte aligned).
 template <typename T>
-__global__ void __launch_bounds__(kWarps * 32)
+__global__ void __launch_bounds__(kWarps * 32, 3)
 step_vec(StepArgs a)
 {
     const int bh = blockIdx.x;

@@ -117,8 +117,8 @@ struct TcParams {
     const float* init;
     __nv_bfloat16* y;
     float* final_state;
-    unsigned int* ctrl;   // [1] CTAs done
-    unsigned int* flags;  // per chain: number of segments published
+    unsigned long long* flags;  // per chain: (epoch, number of segments published)
+    uint32_t epoch;             // tag of this call (see LaunchCtx)
     float* ring;          // per chain: 2 slots of [N][P] fp32
     // Segment-parallel form (chains with many segments): `mode` 1 computes each
     // segment's local end state from zero and its total log2 decay, running only
@@ -702,11 +702,13 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 } else {
                     if (p.mode == 0) {
                         if (n == 0 && !*abort_flag) {
-                            const unsigned int* f = p.flags + s.chain;
+                            const unsigned long long* f = p.flags + s.chain;
                             bool ok = false;
                             const uint64_t t0 = global_timer_ns();
                             for (unsigned long long it = 0; it < p.wait_limit; ++it) {
-                                if (ld_acquire_gpu(f) >= static_cast<unsigned int>(s.seg)) {
+                                const uint64_t v = ld_acquire_gpu_u64(f);
+                                if (static_cast<uint32_t>(v >> 32) == p.epoch &&
+                                    static_cast<uint32_t>(v) >= static_cast<uint32_t>(s.seg)) {
                                     ok = true;
                                     break;
                                 }
@@ -781,7 +783,8 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                         __threadfence();
                         named_bar_sync(kBarOut, 128);
                         if (n == 0 && !p.skip_publish)
-                            st_release_gpu(p.flags + s.chain, static_cast<unsigned int>(s.seg + 1));
+                            st_release_gpu_u64(p.flags + s.chain,
+                                               tagged(p.epoch, static_cast<uint32_t>(s.seg + 1)));
                     }
                 }
             }
@@ -845,16 +848,6 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     tc_fence_before_sync();
     __syncthreads();
     if (warp == kWarpAlloc) tmem_dealloc(tmem, kTmemCols);
-    if (tid == 0) {
-        __threadfence();
-        const unsigned int done = atomicAdd(p.ctrl + 1, 1u);
-        if (done == gridDim.x - 1u) {
-            // every other CTA has finished: leave the control words zeroed
-            for (int c = 0; c < p.chains; ++c) p.flags[c] = 0u;
-            p.ctrl[1] = 0u;
-            __threadfence();
-        }
-    }
 }
 
 // ------------------------------------------------------------------ host side
@@ -957,7 +950,7 @@ WsLayout ws_layout(const FwdArgs& a, const Segments& g)
     const size_t slot = static_cast<size_t>(kP) * kN * sizeof(float);
     w.ctrl = 0;
     w.flags = 256;
-    w.ring = w.flags + ((chains * 4 + 255) / 256) * 256;
+    w.ring = w.flags + ((chains * 8 + 255) / 256) * 256;
     w.total = w.ring + chains * 2 * slot;
     w.seg_state = w.seg_decay = w.seg_hin = w.total;
     if (g.parallel) {
@@ -1016,8 +1009,8 @@ cudaError_t launch(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)
     p.init = a.init;
     p.y = static_cast<__nv_bfloat16*>(a.y);
     p.final_state = a.final_state;
-    p.ctrl = reinterpret_cast<unsigned int*>(ws + w.ctrl);
-    p.flags = reinterpret_cast<unsigned int*>(ws + w.flags);
+    p.flags = reinterpret_cast<unsigned long long*>(ws + w.flags);
+    p.epoch = ctx.epoch;
     p.ring = reinterpret_cast<float*>(ws + w.ring);
     p.seg_state = reinterpret_cast<float*>(ws + w.seg_state);
     p.seg_decay = reinterpret_cast<float*>(ws + w.seg_decay);
@@ -1143,9 +1136,9 @@ extern "C" ssd_status ssd_forward_noalloc(const void* x, const float* dt, const 
                                           int N, int chunk, ssd_dtype dtype, ssd_stream_t stream)
 {
     using namespace ssd;
-    if (B < 0 || L < 0 || H < 1 || G < 1 || P < 1 || N < 1 || chunk < 1 || H % G != 0 ||
-        (dtype != SSD_F32 && dtype != SSD_BF16))
-        return SSD_ERR_INVALID_ARG;
+    // the same size checks as ssd_forward
+    const ssd_status dims = check_dims(B, L, H, P, G, N, chunk, dtype);
+    if (dims != SSD_OK) return dims;
     if ((long long)B * L == 0) return SSD_ERR_UNSUPPORTED;  // nothing for the scratch to do
     if (!x || !dt || !A || !Bm || !Cm || !y) return SSD_ERR_INVALID_ARG;
     const void* ptrs[] = {x, dt, A, Bm, Cm, D, initial_state, y, final_state};
@@ -1178,8 +1171,8 @@ extern "C" ssd_status ssd_forward_noalloc(const void* x, const float* dt, const 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const ssd_status st = acquire_launch_ctx(s, &ctx);
     if (st != SSD_OK) return st;
-    // the ticket, done counter and look-back flags must start at zero
-    if (cudaMemsetAsync(scratch, 0, w.ring, s) != cudaSuccess) return SSD_ERR_CUDA;
+    // nothing in the array needs clearing: the look-back flags carry the tag
+    // of the call that wrote them (see LaunchCtx::epoch)
     const cudaError_t e = tc_forward(a, scratch, ctx);
     return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }

@@ -49,6 +49,8 @@ lib.ssd_set_fault_injection.argtypes = [_i]
 lib.ssd_set_fault_injection.restype = None
 lib.ssd_set_wait_limit.argtypes = [ctypes.c_uint64]
 lib.ssd_set_wait_limit.restype = None
+lib.ssd_set_forward_variant.argtypes = [_i]
+lib.ssd_set_forward_variant.restype = None
 
 SSD_F32, SSD_BF16 = 0, 1
 STATUS = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED",
@@ -123,16 +125,16 @@ def workspace_size(B, L, H, P, G, N, chunk, dtype_code) -> int:
 
 
 def _workspace(device, nbytes: int, stream_handle: int) -> torch.Tensor:
-    """A zero-filled workspace of at least nbytes, cached per (device, stream):
-    calls on one stream are ordered and may share it (the library leaves its
-    control words zeroed after each call); calls on two streams may overlap on
-    the GPU, so each stream gets its own."""
+    """A workspace of at least nbytes, cached per (device, stream): calls on
+    one stream are ordered and may share it (the library tags the control words
+    it keeps there with the call, so no clearing is needed); calls on two
+    streams may overlap on the GPU, so each stream gets its own."""
     dev_index = device.index if device.index is not None else torch.cuda.current_device()
     key = (dev_index, stream_handle)
     with _ws_lock:
         ws = _ws_cache.get(key)
         if ws is None or ws.numel() < nbytes:
-            ws = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
+            ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
             _ws_cache[key] = ws
     return ws
 
@@ -189,7 +191,8 @@ def kernel_count(B, L, H, P, G, N, chunk, dtype_code) -> int:
 
 def forward_path(B, L, H, P, G, N, chunk, dtype_code) -> int:
     """Path of one forward call with these sizes (host-side query): 0 invalid or
-    empty, 1 SIMT, 2 tensor-core single pass, 3 tensor-core segment-parallel."""
+    empty, 1 SIMT, 2 per-head tensor-core single pass, 3 its segment-parallel
+    form, 4 head-group tensor-core kernel."""
     return int(lib.ssd_forward_path(B, L, H, P, G, N, chunk, dtype_code))
 
 
@@ -279,3 +282,9 @@ def set_wait_limit(iterations: int) -> None:
 def set_fault_injection(skip_publish: bool) -> None:
     """Test hook: tiles stop publishing end states (see include/ssd.h)."""
     lib.ssd_set_fault_injection(1 if skip_publish else 0)
+
+
+def set_forward_variant(variant: int) -> None:
+    """Test hook: 0 automatic, 1 per-head tensor-core kernel, 2 head-group
+    tensor-core kernel (see include/ssd.h)."""
+    lib.ssd_set_forward_variant(int(variant))

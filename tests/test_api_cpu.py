@@ -37,10 +37,12 @@ def test_library_exports_every_declared_entry_point(lib):
 
 
 def test_forward_path_query(lib):
-    # bf16 with P = 64 and N a multiple of 8 up to 256 takes the tensor-core
-    # path; few chains on a long sequence run segment-parallel; fp32 and other
-    # sizes take the SIMT path
-    assert lib.ssd_forward_path(4, 4096, 80, 64, 1, 128, 256, 1) == 2
+    # bf16 with P = 64 and N a multiple of 8 up to 256 takes a tensor-core
+    # path: the head-group kernel when there are enough (batch, head pair)
+    # chains and N <= 128, else the per-head kernel; few chains on a long
+    # sequence run segment-parallel; fp32 and other sizes take the SIMT path
+    assert lib.ssd_forward_path(4, 4096, 80, 64, 1, 128, 256, 1) == 4
+    assert lib.ssd_forward_path(8, 2048, 32, 64, 1, 128, 256, 1) == 4
     assert lib.ssd_forward_path(1, 4096, 4, 64, 1, 128, 256, 1) == 3
     assert lib.ssd_forward_path(1, 64, 2, 8, 1, 8, 16, 0) == 1
     assert lib.ssd_forward_path(1, 512, 2, 64, 1, 256, 128, 1) == 2   # N = 256: two passes
@@ -62,12 +64,13 @@ def test_kernel_count_query(lib):
 
 
 def test_workspace_size_formula(lib):
-    """Single pass: 256 B of control words, one 4-byte flag per chain rounded up
-    to 256 B, and a two-slot [128][64] fp32 state ring per chain, where a chain
-    is one 64-channel head slice of one batch row (M = B*H*P/64); the query adds
-    256 bytes of slack."""
+    """Per-head kernel's single pass (the larger of the two tensor-core
+    layouts): 256 B of control words, one 8-byte tagged flag per chain rounded
+    up to 256 B, and a two-slot [128][64] fp32 state ring per chain, where a
+    chain is one 64-channel head slice of one batch row (M = B*H*P/64); the
+    query adds 256 bytes of slack."""
     def single(M):
-        return 256 + (4 * M + 255) // 256 * 256 + M * 2 * 64 * 128 * 4 + 256
+        return 256 + (8 * M + 255) // 256 * 256 + M * 2 * 64 * 128 * 4 + 256
     assert lib.ssd_workspace_size(4, 4096, 80, 64, 1, 128, 256, 1) == single(4 * 80)
     assert lib.ssd_workspace_size(8, 2048, 32, 64, 1, 128, 256, 1) == single(8 * 32)
     assert lib.ssd_workspace_size(2, 8192, 64, 64, 8, 256, 256, 1) == single(2 * 64)  # two passes share it
@@ -78,7 +81,7 @@ def test_segment_parallel_workspace_adds_per_segment_states(lib):
     # long context: 32 chains of 512 tiles; with 148 SMs (the value assumed
     # without a GPU) each chain is cut into 37 segments of 14 tiles
     M, nseg = 32, 37
-    base = 256 + 256 + M * 2 * 64 * 128 * 4 + 256  # control, flags, ring, slack
+    base = 256 + 256 + M * 2 * 64 * 128 * 4 + 256  # control, flags (8 B each), ring, slack
     slot = 64 * 128 * 4
     extra = M * nseg * slot + (4 * M * nseg + 255) // 256 * 256 + M * nseg * slot
     assert lib.ssd_forward_path(1, 65536, 32, 64, 1, 128, 256, 1) == 3
@@ -87,9 +90,10 @@ def test_segment_parallel_workspace_adds_per_segment_states(lib):
 
 
 def test_benchmark_workloads_take_the_tensor_core_path(lib):
-    assert lib.ssd_forward_path(4, 4096, 80, 64, 1, 128, 256, 1) == 2      # 2.7B layer
+    # the layers with many (batch, head pair) chains take the head-group kernel
+    assert lib.ssd_forward_path(4, 4096, 80, 64, 1, 128, 256, 1) == 4      # 2.7B layer
     assert lib.ssd_forward_kernel_count(4, 4096, 80, 64, 1, 128, 256, 1) == 1
-    assert lib.ssd_forward_path(8, 2048, 32, 64, 1, 128, 256, 1) == 2      # 370M layer
+    assert lib.ssd_forward_path(8, 2048, 32, 64, 1, 128, 256, 1) == 4      # 370M layer
     for N in (16, 32, 64, 128, 256):                                       # sweep
         for Q in (128, 256):
             assert lib.ssd_forward_path(2, 8192, 64, 64, 8, N, Q, 1) == 2

@@ -10,7 +10,7 @@ import numpy as np
 import pytest
 
 from selective_state_space_17_b200 import inputs as gen
-from ssd_testutil import TOL, slice_rel_err, to_device, to_host_f64
+from ssd_testutil import TOL, elementwise_rel_err, slice_rel_err, to_device, to_host_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -34,13 +34,17 @@ def _run(ssd, inp, chunk, init=None, D=True):
     return to_host_f64(y), to_host_f64(fs)
 
 
-def _full_check(ssd, oracle, inp, chunk, init=None, D=True):
+def _full_check(ssd, oracle, inp, chunk, init=None, D=True, record=None):
     y, fs = _run(ssd, inp, chunk, init, D)
     x, dt, A, Bm, Cm, Dv = inp.f64()
     yr, fsr = oracle.forward(x, dt, A, Bm, Cm, Dv if D else None, init_state=init)
     tol = TOL[inp.dtype]
     ey = slice_rel_err(y, yr, head_axis=2)
     es = slice_rel_err(fs, fsr, head_axis=1)
+    if record is not None:  # the metric and the elementwise diagnostic, for the record
+        record("slice_rel_err_y", ey)
+        record("slice_rel_err_final_state", es)
+        record("elementwise_rel_err_y", elementwise_rel_err(y, yr))
     assert ey < tol and es < tol, (ey, es)
     return ey, es
 
@@ -58,8 +62,8 @@ def test_tiny_fp32_workload(ssd, oracle):
     ((2, 64, 2, 64, 1, 128), 64),
     ((1, 300, 2, 16, 2, 16), 1),     # chunk of one token
 ])
-def test_fp32_small_shapes(ssd, oracle, shape, chunk):
-    _full_check(ssd, oracle, gen.make_inputs(*shape, "f32", seed=3), chunk)
+def test_fp32_small_shapes(ssd, oracle, shape, chunk, record_property):
+    _full_check(ssd, oracle, gen.make_inputs(*shape, "f32", seed=3), chunk, record=record_property)
 
 
 @pytest.mark.parametrize("shape,chunk", [
@@ -70,8 +74,8 @@ def test_fp32_small_shapes(ssd, oracle, shape, chunk):
     ((1, 512, 2, 64, 1, 16), 128),   # N = 16
     ((1, 130, 3, 24, 3, 40), 48),    # SIMT path in bf16 (P, N off the fast path)
 ])
-def test_bf16_small_shapes(ssd, oracle, shape, chunk):
-    _full_check(ssd, oracle, gen.make_inputs(*shape, "bf16", seed=4), chunk)
+def test_bf16_small_shapes(ssd, oracle, shape, chunk, record_property):
+    _full_check(ssd, oracle, gen.make_inputs(*shape, "bf16", seed=4), chunk, record=record_property)
 
 
 @pytest.mark.parametrize("kind", ["linear_attention", "retnet", "zero_decay"])
