@@ -52,6 +52,15 @@ struct LaunchCtx {
     // of any path or size left there reads as not yet written: a workspace
     // needs no clearing, before its first use or between calls.
     uint32_t epoch;
+
+    // Tag of the i-th launch of this call (i < 8): each launch of a call that
+    // runs several (two passes over the state columns) keeps its own tag, so
+    // it never reads the flags an earlier launch of the same call set.
+    __host__ __device__ uint32_t launch_tag(int i) const
+    {
+        const uint32_t t = epoch * 8u + static_cast<uint32_t>(i);
+        return t ? t : 1u;
+    }
 };
 
 // Control word of this call: (epoch, count).
@@ -60,18 +69,27 @@ __host__ __device__ __forceinline__ unsigned long long tagged(uint32_t epoch, ui
     return (static_cast<unsigned long long>(epoch) << 32) | count;
 }
 
-// Takes the next value of a per-call counter kept as a tagged word: the first
-// taker of a call finds another call's tag (or garbage) and restarts the count
-// at 0 for this call.
+// Takes the next value of a per-call counter. The word holds the count in
+// its high half and the call's tag in its low half, so the common case is one
+// atomicAdd (an add never carries into the tag). The first takers of a call
+// find another call's tag (or garbage): one of them installs this call's tag
+// with count 1 and keeps ticket 0, the others see the new tag and add again.
+// Unlike a compare-and-swap loop, every call costs a bounded number of round
+// trips to L2, however many CTAs take their ticket at the same moment.
 __device__ __forceinline__ unsigned int take_ticket(unsigned long long* ctr, uint32_t epoch)
 {
-    unsigned long long cur = atomicAdd(ctr, 0ull);
+    constexpr unsigned long long kOne = 1ull << 32;
+    unsigned long long old = atomicAdd(ctr, kOne);
     for (;;) {
-        const bool mine = static_cast<uint32_t>(cur >> 32) == epoch;
-        const unsigned long long want = mine ? cur + 1ull : tagged(epoch, 1u);
-        const unsigned long long prev = atomicCAS(ctr, cur, want);
-        if (prev == cur) return mine ? static_cast<unsigned int>(cur) : 0u;
-        cur = prev;
+        if (static_cast<uint32_t>(old) == epoch) return static_cast<unsigned int>(old >> 32);
+        unsigned long long cur = old + kOne;  // the word after our add, if no one else added
+        for (;;) {
+            const unsigned long long prev = atomicCAS(ctr, cur, kOne | epoch);
+            if (prev == cur) return 0u;
+            if (static_cast<uint32_t>(prev) == epoch) break;  // installed by another taker
+            cur = prev;
+        }
+        old = atomicAdd(ctr, kOne);
     }
 }
 

@@ -125,7 +125,7 @@ struct Smem {
     static constexpr uint32_t kHp = kX + 4 * kHalf;      // KH x 16 KB: H' (exact form: raw X)
     static constexpr uint32_t kRec = kHp + 2 * kHalf;    // 2 records
     static constexpr uint32_t kSched = kRec + 2 * sizeof(Rec);
-    static constexpr uint32_t kBars = kSched + 16;
+    static constexpr uint32_t kBars = kSched + 16 * 4;  // kSchedSlots pieces of 16 bytes
     static constexpr int kNumBars = 48;
     static constexpr uint32_t kTmemPtr = kBars + kNumBars * 8;
     static constexpr uint32_t kAbort = kTmemPtr + 4;
@@ -138,7 +138,7 @@ enum Bar : int {
     kEmptyCB = 2,     // 2 (states, MMA3)
     kFullX = 4,       // 2 (tx)
     kEmptyX = 6,      // 2 (states, MMA2, the TMA store of y)
-    kXpFull = 8,      // 2 (four output warps)
+    kXpFull = 8,      // 2 (one per prologue warp)
     kRecFull = 10,    // 2 (one per prologue warp)
     kRecEmpty = 12,   // 2 (MMA B, four state and four output warps)
     kSFull = 14,      // 2
@@ -172,8 +172,9 @@ uint32_t bar_count(int i, int kh)
     if (i == kRecFull || i == kRecFull + 1 || i == kHx) return kh;
     if (i == kRecEmpty || i == kRecEmpty + 1) return 9;
     if (i == kTrilFull || i == kTrilFull + 1 || i == kZEmpty || i == kSlotFull || i == kHReady ||
-        i == kHpFull || i == kZScaled || i == kPub || i == kXpFull || i == kXpFull + 1 || i == kYStaged)
+        i == kHpFull || i == kZScaled || i == kPub || i == kYStaged)
         return 4;
+    if (i == kXpFull || i == kXpFull + 1) return kh;
     if (i >= kSchedEmpty && i < kSchedEmpty + kSchedSlots) return kSchedConsumers;
     return 1;
 }
@@ -203,6 +204,8 @@ struct GParams {
     int gpr;   // head groups per batch row (Ht / KH)
     int hpg;   // kP-channel heads per B/C group (Ht / G)
     int ntiles, chains, seg_len, nseg, items;
+    int wrap;     // 1: static ranges of the chain-major tile order (see Pieces)
+    int grid;
     int skip_publish;
 };
 
@@ -268,46 +271,99 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity)
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
-// A segment of one chain: its batch row, head group and tiles.
+// A piece of one chain: its batch row, head group and tiles [tile_begin,
+// tile_end). `seg` counts the pieces of the chain before this one: a piece
+// with seg > 0 starts from the state its predecessor published.
 struct Pos {
-    int item, seg, chain, b, hs0, g, tile, tile_end;
+    int chain, seg, b, hs0, g, tile, tile_begin, tile_end;
     bool valid;
 
-    __device__ __noinline__ void decode(const GParams& p, int it, int kh)
+    __device__ void set(const GParams& p, int4 pc, int kh)
     {
-        item = it;
-        valid = it >= 0 && it < p.items;
+        valid = pc.x >= 0;
         if (!valid) return;
-        seg = it / p.chains;
-        chain = it - seg * p.chains;
+        chain = pc.x;
+        seg = pc.y;
+        tile_begin = tile = pc.z;
+        tile_end = pc.w;
         b = chain / p.gpr;
         hs0 = (chain - b * p.gpr) * kh;
         g = hs0 / p.hpg;
-        tile = seg * p.seg_len;
-        tile_end = min(tile + p.seg_len, p.ntiles);
     }
 };
 
-// Ticket ring: the producer pushes segment numbers, warps 1..12 read each one.
+// The pieces one CTA runs, in order.
+//  Segment mode: ticket t is segment t / chains of chain t % chains (segments
+//  of seg_len tiles, numbered segment-major, so a segment's predecessor was
+//  taken by a CTA that was already running).
+//  Wrap mode (at least as many chains as CTAs): one ticket per CTA gives its
+//  rank c, which owns tiles [c U / grid, (c+1) U / grid) of the chain-major
+//  order of all U tiles. That range is the tail of one chain, whole chains and
+//  the head of another; the CTA runs the head first and the tail last. The
+//  head's other part is the tail of rank c + 1, which runs it last, so it
+//  waits on a piece that a running CTA does first, with a slack of
+//  U / grid - ntiles tiles (the range is at least one chain long).
+struct Pieces {
+    long long u0 = 0, u1 = 0;
+    int idx = 0;
+    __device__ int4 next(const GParams& p, volatile int* abort_flag)
+    {
+        const int4 none = make_int4(-1, 0, 0, 0);
+        if (*abort_flag) return none;
+        if (!p.wrap) {
+            const unsigned int t = take_ticket(p.ctrl, p.epoch);
+            if (t >= static_cast<unsigned int>(p.items)) return none;
+            const int seg = static_cast<int>(t) / p.chains;
+            const int tb = seg * p.seg_len;
+            return make_int4(static_cast<int>(t) - seg * p.chains, seg, tb, min(tb + p.seg_len, p.ntiles));
+        }
+        const long long U = static_cast<long long>(p.chains) * p.ntiles;
+        if (idx == 0) {
+            const unsigned int c = take_ticket(p.ctrl, p.epoch);
+            if (c >= static_cast<unsigned int>(p.grid)) return none;
+            u0 = c * U / p.grid;
+            u1 = (c + 1ll) * U / p.grid;
+        }
+        const int nt = p.ntiles;
+        const int ca = static_cast<int>(u0 / nt), oa = static_cast<int>(u0 % nt);
+        const int cb = static_cast<int>(u1 / nt), ob = static_cast<int>(u1 % nt);
+        const int first_full = oa > 0 ? ca + 1 : ca;
+        int j = idx++;
+        if (ob > 0) {
+            if (j == 0) return make_int4(cb, 0, 0, ob);  // head of chain cb
+            --j;
+        }
+        if (first_full + j < cb) return make_int4(first_full + j, 0, 0, nt);
+        j -= cb - first_full;
+        if (oa > 0 && j == 0) return make_int4(ca, 1, oa, nt);  // tail of chain ca
+        return none;
+    }
+};
+
+// Piece ring: the producer pushes pieces, warps 1..12 read each one.
 struct SchedReader {
     uint32_t n = 0;
     // Every reader sees the same sequence (the producer never overwrites an
-    // unread slot and pushes -1 to end it), so the warps of one role walk the
+    // unread slot and pushes an end marker), so the warps of one role walk the
     // same tiles. A reader that waits in vain (the producer is gone) ends its
     // sequence after the bounded wait; in abort mode every reader ends at once
     // (the roles are linked by mbarriers only, so no role waits on a warp
     // that has left its loop for longer than a bounded wait).
-    __device__ int pop(uint8_t* sm, uint64_t* bars, volatile int* abort_flag, unsigned int* status)
+    __device__ int4 pop(uint8_t* sm, uint64_t* bars, volatile int* abort_flag, unsigned int* status)
     {
-        if (*abort_flag) return -1;  // aborted: the results are undefined, every role just ends
+        if (*abort_flag) return make_int4(-1, 0, 0, 0);  // aborted: every role just ends
         const uint32_t slot = n % kSchedSlots;
         const bool ok = wait_bounded(bars + kSchedFull + slot, (n / kSchedSlots) & 1);
-        const int it = ok ? *reinterpret_cast<volatile int*>(sm + Smem::kSched + slot * 4) : -1;
+        int4 pc = make_int4(-1, 0, 0, 0);
+        if (ok) {
+            const volatile int* v = reinterpret_cast<const volatile int*>(sm + Smem::kSched + slot * 16);
+            pc = make_int4(v[0], v[1], v[2], v[3]);
+        }
         if (!ok && (threadIdx.x & 31) == 0) wait_gave_up(abort_flag, status);
         __syncwarp();
         if ((threadIdx.x & 31) == 0) mbar_arrive(bars + kSchedEmpty + slot);
         ++n;
-        return it;
+        return pc;
     }
 };
 
@@ -317,11 +373,11 @@ struct Walker {
     SchedReader rd;
     __device__ void begin(const GParams& p, uint8_t* sm, uint64_t* bars, volatile int* ab)
     {
-        s.decode(p, rd.pop(sm, bars, ab, p.status), KH);
+        s.set(p, rd.pop(sm, bars, ab, p.status), KH);
     }
     __device__ void next(const GParams& p, uint8_t* sm, uint64_t* bars, volatile int* ab)
     {
-        if (++s.tile >= s.tile_end) s.decode(p, rd.pop(sm, bars, ab, p.status), KH);
+        if (++s.tile >= s.tile_end) s.set(p, rd.pop(sm, bars, ab, p.status), KH);
     }
 };
 
@@ -382,15 +438,17 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
         // Tickets are taken one segment ahead, so that the L2 prefetch of the
         // tiles kPrefetch ahead runs across segment boundaries too.
         uint32_t npush = 0;
+        Pieces src;
         auto fetch = [&]() {
-            int it = -1;
-            if (lane == 0 && !*abort_flag) {
-                const unsigned int t = take_ticket(p.ctrl, p.epoch);
-                it = t < static_cast<unsigned int>(p.items) ? static_cast<int>(t) : -1;
-            }
-            return __shfl_sync(0xffffffffu, it, 0);
+            int4 pc = make_int4(-1, 0, 0, 0);
+            if (lane == 0) pc = src.next(p, abort_flag);
+            pc.x = __shfl_sync(0xffffffffu, pc.x, 0);
+            pc.y = __shfl_sync(0xffffffffu, pc.y, 0);
+            pc.z = __shfl_sync(0xffffffffu, pc.z, 0);
+            pc.w = __shfl_sync(0xffffffffu, pc.w, 0);
+            return pc;
         };
-        auto push = [&](int it) {
+        auto push = [&](int4 pc) {
             if (*abort_flag) return false;  // the readers end at once in abort mode
             const uint32_t slot = npush % kSchedSlots;
             // never overwrite a slot a reader has not taken yet, even when aborting
@@ -400,7 +458,11 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
                 return false;
             }
             if (lane == 0) {
-                *reinterpret_cast<volatile int*>(sm + Smem::kSched + slot * 4) = it;
+                volatile int* v = reinterpret_cast<volatile int*>(sm + Smem::kSched + slot * 16);
+                v[0] = pc.x;
+                v[1] = pc.y;
+                v[2] = pc.z;
+                v[3] = pc.w;
                 mbar_arrive(bars + kSchedFull + slot);
             }
             __syncwarp();
@@ -416,10 +478,14 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
 #pragma unroll
             for (int hh = 0; hh < KH; ++hh) tma_prefetch_l2_4d(&tmX, 0, q.hs0 + hh, t0, q.b);
         };
+        const int4 kEnd = make_int4(-1, 0, 0, 0);
         Pos s, nx;
-        s.decode(p, fetch(), KH);
-        bool alive = push(s.valid ? s.item : -1);
-        nx.decode(p, s.valid ? fetch() : -1, KH);
+        int4 pc = fetch();
+        s.set(p, pc, KH);
+        bool alive = push(pc);
+        pc = s.valid ? fetch() : kEnd;
+        nx.set(p, pc, KH);
+        int4 pc_nx = pc;
         int k = 0;
         if (s.valid && elect_one_sync()) {
             // the tiles before the prefetch distance
@@ -465,11 +531,12 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             ++k;
             if (++s.tile >= s.tile_end) {
                 s = nx;
-                alive = push(s.valid ? s.item : -1);
-                nx.decode(p, s.valid ? fetch() : -1, KH);
+                alive = push(pc_nx);
+                pc_nx = s.valid ? fetch() : kEnd;
+                nx.set(p, pc_nx, KH);
             }
         }
-        if (alive && s.valid) push(-1);  // aborted: tell every role to stop
+        if (alive && s.valid) push(kEnd);  // aborted: tell every role to stop
         // every load issued has landed before the CTA can exit
         for (int j = max(0, k - 2); j < k; ++j) {
             wait_bounded(bars + kFullCB + (j & 1), (j >> 1) & 1);
@@ -612,7 +679,7 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
         __syncwarp();
         wait_bounded(bars + kDrainB, 0);
     } else if (warp == kWarpPro0 || warp == kWarpPro1) {
-        // ---------------------------------------- prologue: decay, record (one head)
+        // ------------------------------------ prologue: decay, record, X' (one head)
         const int hh = warp == kWarpPro0 ? 0 : 1;
         Walker<KH> w;
         w.begin(p, sm, bars, abort_flag);
@@ -676,6 +743,29 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bars + kRecFull + st);
+
+                // X' = diag(f) X in place (fp32 product, one rounding). Chunk c of
+                // the head's tile (16 bytes) is in row c / 8 whatever the swizzle
+                // does inside the row; the factor of row j comes from lane j % 32.
+                float f[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    f[u] = ex2_approx(hard ? cs_end - cs[u] : cref - cs[u]) * dtc[u];
+                wait_bar(bars + kFullX + st, par, abort_flag, p.status);
+                uint4* xt = reinterpret_cast<uint4*>(sm + Smem::kX + st * 2 * kHalf + hh * kHalf);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int c = j * 32 + lane;
+                    const float fr = __shfl_sync(0xffffffffu, f[j >> 3], (c >> 3) & 31);
+                    const uint4 v = xt[c];
+                    xt[c] = make_uint4(pack_bf16x2(fr * bf16_lo(v.x), fr * bf16_hi(v.x)),
+                                       pack_bf16x2(fr * bf16_lo(v.y), fr * bf16_hi(v.y)),
+                                       pack_bf16x2(fr * bf16_lo(v.z), fr * bf16_hi(v.z)),
+                                       pack_bf16x2(fr * bf16_lo(v.w), fr * bf16_hi(v.w)));
+                }
+                fence_async_shared();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bars + kXpFull + st);
             }
         } else {
             while (w.s.valid) w.next(p, sm, bars, abort_flag);  // KH = 1: read the tickets only
@@ -706,30 +796,26 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
                 tc_fence_after_sync();
                 if (prev_last) {
                     const bool fin = prev.tile == p.ntiles - 1;
-#pragma unroll
-                    for (int hh = 0; hh < KH; ++hh) {
 #pragma unroll 1
-                        for (int half = 0; half < 2; ++half) {
-                            float v[32];
-                            tmem_ld32(tmem + lane_off + kColH + hh * 64 + half * 32, v);
-                            tmem_wait_ld();
-                            if (fin) {
-                                if (p.final_state && n_live) {
-                                    float* dst = p.final_state +
-                                                 ((static_cast<size_t>(prev.b) * p.Ht + prev.hs0 + hh) * kP +
-                                                  half * 32) * Nst + r;
+                    for (int hh = 0; hh < KH; ++hh) {
+                        uint32_t v[64];
+                        tmem_ld64_sync(tmem + lane_off + kColH + hh * 64, v);
+                        const float sp = s_pend[hh];
+                        if (fin) {
+                            if (p.final_state && n_live) {
+                                float* dst = p.final_state +
+                                             (static_cast<size_t>(prev.b) * p.Ht + prev.hs0 + hh) * kP * Nst + r;
 #pragma unroll
-                                    for (int q = 0; q < 32; ++q) dst[q * Nst] = s_pend[hh] * v[q];
-                                }
-                            } else {
-                                float4* dst = reinterpret_cast<float4*>(
-                                    p.ring + ((static_cast<size_t>(prev.chain) * KH + hh) * kN + r) * kP +
-                                    half * 32);
-#pragma unroll
-                                for (int q = 0; q < 8; ++q)
-                                    dst[q] = make_float4(s_pend[hh] * v[4 * q], s_pend[hh] * v[4 * q + 1],
-                                                         s_pend[hh] * v[4 * q + 2], s_pend[hh] * v[4 * q + 3]);
+                                for (int q = 0; q < 64; ++q) dst[q * Nst] = sp * __uint_as_float(v[q]);
                             }
+                        } else {
+                            float4* dst = reinterpret_cast<float4*>(
+                                p.ring + ((static_cast<size_t>(prev.chain) * KH + hh) * kN + r) * kP);
+#pragma unroll
+                            for (int q = 0; q < 16; ++q)
+                                dst[q] = make_float4(sp * __uint_as_float(v[4 * q]), sp * __uint_as_float(v[4 * q + 1]),
+                                                     sp * __uint_as_float(v[4 * q + 2]),
+                                                     sp * __uint_as_float(v[4 * q + 3]));
                         }
                     }
                     if (!fin) {
@@ -766,7 +852,7 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
                 snext[hh] = hard ? 1.f : ex2_approx(ce - c);
             }
             // ---- H' (bf16 operand of MMA3) and the scaled state for tile k
-            const bool first = w.s.tile == w.s.seg * p.seg_len;
+            const bool first = w.s.tile == w.s.tile_begin;
             if (first && w.s.seg > 0) {
                 // bounded acquire poll on the predecessor's flag, one per warp.
                 // Giving up only records the status: the call's results are
@@ -795,51 +881,45 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             for (int hh = 0; hh < KH; ++hh) {
                 if (first) s_pend[hh] = 1.f;
                 const float f3 = sig3[hh] * s_pend[hh], fst = sigst[hh] * s_pend[hh];
-#pragma unroll 1
-                for (int half = 0; half < 2; ++half) {
-                    float v[32];
-                    const uint32_t a = tmem + lane_off + kColH + hh * 64 + half * 32;
-                    if (!first) {
-                        tmem_ld32(a, v);
-                        tmem_wait_ld();
-                    } else if (w.s.seg > 0) {
-                        // what the predecessor published: row r of [kN][kP]
-                        const float4* src = reinterpret_cast<const float4*>(
-                            p.ring + ((static_cast<size_t>(w.s.chain) * KH + hh) * kN + r) * kP + half * 32);
+                const uint32_t a = tmem + lane_off + kColH + hh * 64;
+                uint32_t v[64];  // fp32 bits of row r of this head's h
+                if (!first) {
+                    tmem_ld64_sync(a, v);
+                } else if (w.s.seg > 0) {
+                    // what the predecessor published: row r of [kN][kP]
+                    const float4* src = reinterpret_cast<const float4*>(
+                        p.ring + ((static_cast<size_t>(w.s.chain) * KH + hh) * kN + r) * kP);
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            const float4 u = __ldcg(src + q);
-                            v[4 * q] = u.x;
-                            v[4 * q + 1] = u.y;
-                            v[4 * q + 2] = u.z;
-                            v[4 * q + 3] = u.w;
-                        }
-                    } else if (p.init && n_live) {
-                        // the chain's initial state, [B][H][P][N]
-                        const float* src = p.init +
-                                           ((static_cast<size_t>(w.s.b) * p.Ht + w.s.hs0 + hh) * kP + half * 32) *
-                                               Nst + r;
-#pragma unroll
-                        for (int q = 0; q < 32; ++q) v[q] = __ldg(src + q * Nst);
-                    } else {
-#pragma unroll
-                        for (int q = 0; q < 32; ++q) v[q] = 0.f;
+                    for (int q = 0; q < 16; ++q) {
+                        const float4 u = __ldcg(src + q);
+                        v[4 * q] = __float_as_uint(u.x);
+                        v[4 * q + 1] = __float_as_uint(u.y);
+                        v[4 * q + 2] = __float_as_uint(u.z);
+                        v[4 * q + 3] = __float_as_uint(u.w);
                     }
-                    uint8_t* row = sm + Smem::kHp + hh * kHalf + r * 128;
+                } else if (p.init && n_live) {
+                    // the chain's initial state, [B][H][P][N]
+                    const float* src = p.init + (static_cast<size_t>(w.s.b) * p.Ht + w.s.hs0 + hh) * kP * Nst + r;
 #pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) {
-                        const int chunk = half * 4 + cc;
-                        const uint4 hv = make_uint4(pack_bf16x2(f3 * v[cc * 8 + 0], f3 * v[cc * 8 + 1]),
-                                                    pack_bf16x2(f3 * v[cc * 8 + 2], f3 * v[cc * 8 + 3]),
-                                                    pack_bf16x2(f3 * v[cc * 8 + 4], f3 * v[cc * 8 + 5]),
-                                                    pack_bf16x2(f3 * v[cc * 8 + 6], f3 * v[cc * 8 + 7]));
-                        *reinterpret_cast<uint4*>(row + (((chunk ^ r) & 7) << 4)) = hv;
-                    }
-                    uint32_t o[32];
+                    for (int q = 0; q < 64; ++q) v[q] = __float_as_uint(__ldg(src + q * Nst));
+                } else {
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(fst * v[q]);
-                    tmem_st32(a, o);
+                    for (int q = 0; q < 64; ++q) v[q] = 0u;
                 }
+                uint8_t* row = sm + Smem::kHp + hh * kHalf + r * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint32_t* u = v + c * 8;
+                    const uint4 hv = make_uint4(
+                        pack_bf16x2(f3 * __uint_as_float(u[0]), f3 * __uint_as_float(u[1])),
+                        pack_bf16x2(f3 * __uint_as_float(u[2]), f3 * __uint_as_float(u[3])),
+                        pack_bf16x2(f3 * __uint_as_float(u[4]), f3 * __uint_as_float(u[5])),
+                        pack_bf16x2(f3 * __uint_as_float(u[6]), f3 * __uint_as_float(u[7])));
+                    *reinterpret_cast<uint4*>(row + (((c ^ r) & 7) << 4)) = hv;
+                }
+#pragma unroll
+                for (int q = 0; q < 64; ++q) v[q] = __float_as_uint(fst * __uint_as_float(v[q]));
+                tmem_st64(a, v);
                 s_pend[hh] = snext[hh];
             }
             tmem_wait_st();
@@ -857,24 +937,29 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             wait_bar(bars + kSFull + st, par, abort_flag, p.status);
             tc_fence_after_sync();
             const uint32_t s_col = tmem + lane_off + kColS + st * 128;
+            // rows of lane quadrant wq need S blocks jb <= wq: blocks (0, 1) and
+            // (2, 3) are read as 64-column pairs, and each pair's bf16 output
+            // (32 columns at 32 jp) covers only columns read before
 #pragma unroll 1
-            for (int jb = 0; jb < 4; ++jb) {
-                uint32_t packed[16];
-                if (jb <= wq) {
-                    float sv[32];
-                    tmem_ld32(s_col + jb * 32, sv);
-                    tmem_wait_ld();
-                    if (jb == wq) {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) sv[e] = e <= lane ? sv[e] : 0.f;
-                    }
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) packed[q] = pack_bf16x2(sv[2 * q], sv[2 * q + 1]);
+            for (int jp = 0; jp < 2; ++jp) {
+                uint32_t sv[64];
+                if (2 * jp <= wq) {
+                    tmem_ld64_sync(s_col + jp * 64, sv);
                 } else {
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) packed[q] = 0u;
+                    for (int e = 0; e < 64; ++e) sv[e] = 0u;
                 }
-                tmem_st16(s_col + jb * 16, packed);
+                // packed in place: word q takes values 2q, 2q + 1 (never behind q)
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    const int e = 2 * q, jb = 2 * jp + (e >> 5), c = e & 31;
+                    // keep j <= i: blocks left of the diagonal whole, the
+                    // diagonal block up to column lane, nothing to the right
+                    const float s0 = (jb < wq || (jb == wq && c <= lane)) ? __uint_as_float(sv[e]) : 0.f;
+                    const float s1 = (jb < wq || (jb == wq && c + 1 <= lane)) ? __uint_as_float(sv[e + 1]) : 0.f;
+                    sv[q] = pack_bf16x2(s0, s1);
+                }
+                tmem_st32(s_col + jp * 32, sv);
             }
             tmem_wait_st();
             tc_fence_before_sync();
@@ -932,172 +1017,121 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             w.next(p, sm, bars, abort_flag);
         }
     } else if (warp >= kWgOut && warp < kWgOut + 4) {
-        // -------------------------- output: X' in place, then y = e Z + D x.
-        // Thread r owns token row r of a tile: it writes X'_r = f_r x_r over
-        // the row of x, and later y_r over X'_r, taking x_r for the D term back
-        // as X'_r / f_r (one more bf16 rounding of that term), or from global
-        // memory where f_r is too small for that (dt_r = 0, or an early token
-        // of an exact-form tile); one TMA store per head then writes the tile
-        // (rows past L are clipped). X' of tile k + 1 is built before the
-        // output of tile k, so that its products are not held up by the
-        // output. Exact form: first Z_r *= 2^(cs_r), which the per-head
+        // ------------------------------------------- output: y = e Z + D x.
+        // Thread r owns token row r of the tile and writes y_r over the row
+        // X'_r of the X stage, taking x_r for the D term back as X'_r / f_r (one
+        // more bf16 rounding of that term), or from global memory where f_r is
+        // too small for that (dt_r = 0, or an early token of an exact-form
+        // tile); one TMA store per head then writes the tile (rows past L are
+        // clipped), and the stage goes back to the producer once the stores
+        // have read it. Exact form: first Z_r *= 2^(cs_r), which the per-head
         // masked products then add to.
         const int wq = warp - kWgOut;
         const int r = wq * 32 + lane;  // token row i = TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-        struct TileOut {
-            Pos pos;
-            float f[KH], e[KH], zs[KH], Dh[KH];
-            bool hard;
-        };
         Walker<KH> w;
         w.begin(p, sm, bars, abort_flag);
-        TileOut cur, nxt;
-        bool have_cur = false;
         uint32_t nh = 0;
-        int k = 0;  // the tile whose output is pending; X' is built for tile k + have_cur
-        for (;;) {
-            const bool have_nx = w.s.valid;
-            if (have_nx) {
-                // ---- X' of the next tile
-                const int kx = k + (have_cur ? 1 : 0);
-                const int st = kx & 1;
-                const uint32_t par = (kx >> 1) & 1;
-                nxt.pos = w.s;
-                const bool live = r < p.L - w.s.tile * kT;
-                float dtr[KH];
+        for (int k = 0; w.s.valid; ++k, w.next(p, sm, bars, abort_flag)) {
+            const Pos cur = w.s;
+            const int st = k & 1;
+            const uint32_t par = (k >> 1) & 1;
+            uint8_t* xs = sm + Smem::kX + st * 2 * kHalf;
+            const bool live = r < p.L - cur.tile * kT;
+            float dtr[KH], Dh[KH];
 #pragma unroll
-                for (int hh = 0; hh < KH; ++hh) {
-                    const int hr = (w.s.hs0 + hh) / p.sub;
-                    dtr[hh] = live ? __ldg(p.dt + (static_cast<size_t>(w.s.b) * p.L + w.s.tile * kT + r) * p.Hr + hr)
-                                   : 0.f;
-                    nxt.Dh[hh] = p.D ? __ldg(p.D + hr) : 0.f;
-                }
-                const Rec& rc = recs[st];
-                wait_bar(bars + kRecFull + st, par, abort_flag, p.status);
-                nxt.hard = rc.hard != 0;
-#pragma unroll
-                for (int hh = 0; hh < KH; ++hh) {
-                    const float ci = rc.cs[hh][r];
-                    nxt.f[hh] = ex2_approx(nxt.hard ? rc.csend[hh] - ci : rc.cref[hh] - ci) * dtr[hh];
-                    nxt.e[hh] = nxt.hard ? 1.f : ex2_approx(ci - rc.cref[hh]);
-                    nxt.zs[hh] = ex2_approx(ci);
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bars + kRecEmpty + st);
-                // X' = diag(f) X in place, in fp32 with one rounding
-                wait_bar(bars + kFullX + st, par, abort_flag, p.status);
-                uint8_t* xs = sm + Smem::kX + st * 2 * kHalf;
-#pragma unroll
-                for (int hh = 0; hh < KH; ++hh) {
-                    uint8_t* row = xs + hh * kHalf + r * 128;
-                    const float fh = nxt.f[hh];
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        uint4* a = reinterpret_cast<uint4*>(row + (((c ^ r) & 7) << 4));
-                        const uint4 v = *a;
-                        *a = make_uint4(pack_bf16x2(fh * bf16_lo(v.x), fh * bf16_hi(v.x)),
-                                        pack_bf16x2(fh * bf16_lo(v.y), fh * bf16_hi(v.y)),
-                                        pack_bf16x2(fh * bf16_lo(v.z), fh * bf16_hi(v.z)),
-                                        pack_bf16x2(fh * bf16_lo(v.w), fh * bf16_hi(v.w)));
-                    }
-                }
-                fence_async_shared();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bars + kXpFull + st);
+            for (int hh = 0; hh < KH; ++hh) {
+                const int hr = (cur.hs0 + hh) / p.sub;
+                dtr[hh] = live ? __ldg(p.dt + (static_cast<size_t>(cur.b) * p.L + cur.tile * kT + r) * p.Hr + hr)
+                               : 0.f;
+                Dh[hh] = p.D ? __ldg(p.D + hr) : 0.f;
             }
-            if (have_cur) {
-                // ---- output of tile k
-                const int st = k & 1;
-                uint8_t* xs = sm + Smem::kX + st * 2 * kHalf;
-                if (cur.hard) {
-                    wait_bar(bars + kM3Done, nh & 1, abort_flag, p.status);
-                    tc_fence_after_sync();
+            const Rec& rc = recs[st];
+            wait_bar(bars + kRecFull + st, par, abort_flag, p.status);
+            const bool hard = rc.hard != 0;
+            float f[KH], e[KH], zs[KH];
 #pragma unroll
-                    for (int hh = 0; hh < KH; ++hh) {
-#pragma unroll 1
-                        for (int qd = 0; qd < 4; ++qd) {
-                            float v[16];
-                            uint32_t o[16];
-                            const uint32_t a = tmem + lane_off + kColZ + hh * 64 + qd * 16;
-                            tmem_ld16(a, v);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int q = 0; q < 16; ++q) o[q] = __float_as_uint(v[q] * cur.zs[hh]);
-                            tmem_st16(a, o);
-                        }
-                    }
-                    tmem_wait_st();
-                    tc_fence_before_sync();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bars + kZScaled);
-                    ++nh;
-                }
-                // y over X' once MMA2 (Z full) and the states MMA have read it.
-                // (A per-stage barrier: the single-phase "states done" could
-                // already have completed for tile k + 1, whose X' is built above.)
-                wait_bar(bars + kZFull, k & 1, abort_flag, p.status);
-                wait_bar(bars + kXRead + st, (k >> 1) & 1, abort_flag, p.status);
+            for (int hh = 0; hh < KH; ++hh) {
+                const float ci = rc.cs[hh][r];
+                f[hh] = ex2_approx(hard ? rc.csend[hh] - ci : rc.cref[hh] - ci) * dtr[hh];
+                e[hh] = hard ? 1.f : ex2_approx(ci - rc.cref[hh]);
+                zs[hh] = ex2_approx(ci);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars + kRecEmpty + st);
+            if (hard) {
+                wait_bar(bars + kM3Done, nh & 1, abort_flag, p.status);
                 tc_fence_after_sync();
-                const bool live = r < p.L - cur.pos.tile * kT;
-#pragma unroll
+#pragma unroll 1
                 for (int hh = 0; hh < KH; ++hh) {
-                    uint8_t* row = xs + hh * kHalf + r * 128;
-                    // D x_r from X'_r / f_r, or from global memory where f_r is tiny
-                    const bool from_xp = cur.f[hh] >= 0x1p-100f;
-                    const float dx = from_xp ? cur.Dh[hh] / cur.f[hh] : cur.Dh[hh];
-                    const uint4* xg = reinterpret_cast<const uint4*>(
-                        p.x + ((static_cast<size_t>(cur.pos.b) * p.L + cur.pos.tile * kT + r) * p.Ht +
-                               cur.pos.hs0 + hh) * kP);
+                    uint32_t v[64];
+                    const uint32_t a = tmem + lane_off + kColZ + hh * 64;
+                    tmem_ld64_sync(a, v);
+                    const float zsh = (KH == 2 && hh) ? zs[KH - 1] : zs[0];
 #pragma unroll
-                    for (int qd = 0; qd < 4; ++qd) {
-                        float zv[16];
-                        tmem_ld16(tmem + lane_off + kColZ + hh * 64 + qd * 16, zv);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int q = 0; q < 2; ++q) {
-                            const int c = qd * 2 + q;
-                            uint4* a = reinterpret_cast<uint4*>(row + (((c ^ r) & 7) << 4));
-                            uint4 xq = *a;
-                            if (!from_xp)
-                                xq = (live && cur.Dh[hh] != 0.f) ? __ldg(xg + c) : make_uint4(0u, 0u, 0u, 0u);
-                            const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
-                            uint32_t o[4];
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                const int j = q * 8 + u * 2;
-                                o[u] = pack_bf16x2(fmaf(cur.e[hh], zv[j], dx * bf16_lo(xw[u])),
-                                                   fmaf(cur.e[hh], zv[j + 1], dx * bf16_hi(xw[u])));
-                            }
-                            *a = make_uint4(o[0], o[1], o[2], o[3]);
-                        }
-                    }
+                    for (int q = 0; q < 64; ++q) v[q] = __float_as_uint(__uint_as_float(v[q]) * zsh);
+                    tmem_st64(a, v);
                 }
+                tmem_wait_st();
                 tc_fence_before_sync();
-                fence_async_shared();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(bars + kZEmpty);
-                    mbar_arrive(bars + kYStaged);
-                }
-                if (r == 0) {
-                    // one TMA store per head once all four warps staged their rows;
-                    // the stage returns to the producer when the stores have read it
-                    wait_bar_1(bars + kYStaged, k & 1, abort_flag, p.status);
-#pragma unroll
-                    for (int hh = 0; hh < KH; ++hh)
-                        tma_store_4d(&tmY, xs + hh * kHalf, 0, cur.pos.hs0 + hh, cur.pos.tile * kT, cur.pos.b);
-                    tma_store_commit();
-                    tma_store_wait_read();
-                    mbar_arrive(bars + kEmptyX + st);
-                }
-                __syncwarp();
-                ++k;
+                if (lane == 0) mbar_arrive(bars + kZScaled);
+                ++nh;
             }
-            if (!have_nx) break;
-            cur = nxt;
-            have_cur = true;
-            w.next(p, sm, bars, abort_flag);
+            // y over X' once MMA2 (Z full) and the states MMA (per-stage barrier)
+            // have read it
+            wait_bar(bars + kZFull, k & 1, abort_flag, p.status);
+            wait_bar(bars + kXRead + st, par, abort_flag, p.status);
+            tc_fence_after_sync();
+#pragma unroll 1
+            for (int hh = 0; hh < KH; ++hh) {
+                uint8_t* row = xs + hh * kHalf + r * 128;
+                // per-head scalars by selection (no indexing by the loop counter)
+                const float fh = (KH == 2 && hh) ? f[KH - 1] : f[0];
+                const float Dhh = (KH == 2 && hh) ? Dh[KH - 1] : Dh[0];
+                const float eh = (KH == 2 && hh) ? e[KH - 1] : e[0];
+                // D x_r from X'_r / f_r, or from global memory where f_r is tiny
+                const bool from_xp = fh >= 0x1p-100f;
+                const float dx = from_xp ? Dhh / fh : Dhh;
+                const uint4* xg = reinterpret_cast<const uint4*>(
+                    p.x + ((static_cast<size_t>(cur.b) * p.L + cur.tile * kT + r) * p.Ht + cur.hs0 + hh) * kP);
+                uint32_t zv[64];
+                tmem_ld64_sync(tmem + lane_off + kColZ + hh * 64, zv);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint4* a = reinterpret_cast<uint4*>(row + (((c ^ r) & 7) << 4));
+                    uint4 xq = *a;
+                    if (!from_xp) xq = (live && Dhh != 0.f) ? __ldg(xg + c) : make_uint4(0u, 0u, 0u, 0u);
+                    const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
+                    uint32_t o[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int j = c * 8 + u * 2;
+                        o[u] = pack_bf16x2(fmaf(eh, __uint_as_float(zv[j]), dx * bf16_lo(xw[u])),
+                                           fmaf(eh, __uint_as_float(zv[j + 1]), dx * bf16_hi(xw[u])));
+                    }
+                    *a = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+            }
+            tc_fence_before_sync();
+            fence_async_shared();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bars + kZEmpty);
+                mbar_arrive(bars + kYStaged);
+            }
+            if (r == 0) {
+                // one TMA store per head once all four warps staged their rows;
+                // the stage returns to the producer when the stores have read it
+                wait_bar_1(bars + kYStaged, k & 1, abort_flag, p.status);
+#pragma unroll
+                for (int hh = 0; hh < KH; ++hh)
+                    tma_store_4d(&tmY, xs + hh * kHalf, 0, cur.hs0 + hh, cur.tile * kT, cur.b);
+                tma_store_commit();
+                tma_store_wait_read();
+                mbar_arrive(bars + kEmptyX + st);
+            }
+            __syncwarp();
         }
         if (r == 0) tma_store_wait_all();
     }
@@ -1118,7 +1152,7 @@ int heads_per_tile(const FwdArgs& a)
 }
 
 struct Plan {
-    int KH, Ht, chains, ntiles, seg_len, nseg, items, grid;
+    int KH, Ht, chains, ntiles, seg_len, nseg, items, grid, wrap;
     size_t ws_ctrl, ws_flags, ws_ring, ws_total;
 };
 
@@ -1132,13 +1166,25 @@ Plan make_plan(const FwdArgs& a, int ctas)
     g.Ht = a.H * (a.P / kP);
     g.chains = a.B * (g.Ht / g.KH);
     g.ntiles = (a.L + kT - 1) / kT;
-    long long want = (static_cast<long long>(kItemsPerCta) * ctas + g.chains - 1) / g.chains;
-    if (want < 1) want = 1;
-    if (want > g.ntiles) want = g.ntiles;
-    g.seg_len = static_cast<int>((g.ntiles + want - 1) / want);
-    g.nseg = (g.ntiles + g.seg_len - 1) / g.seg_len;
-    g.items = g.chains * g.nseg;
-    g.grid = g.items < ctas ? g.items : ctas;
+    g.wrap = 0;
+    if (g.chains >= ctas) {
+        // every CTA owns an equal range of the chain-major tile order, at least
+        // one chain long: at most one hand-off per CTA, none waited on long
+        g.wrap = 1;
+        g.seg_len = g.ntiles;
+        g.nseg = 2;
+        g.items = ctas;
+        g.grid = ctas;
+    } else {
+        long long want = 1;
+        if (g.chains < ctas / 2)  // else one chain per CTA: no hand-offs
+            want = (static_cast<long long>(kItemsPerCta) * ctas + g.chains - 1) / g.chains;
+        if (want > g.ntiles) want = g.ntiles;
+        g.seg_len = static_cast<int>((g.ntiles + want - 1) / want);
+        g.nseg = (g.ntiles + g.seg_len - 1) / g.seg_len;
+        g.items = g.chains * g.nseg;
+        g.grid = g.items < ctas ? g.items : ctas;
+    }
     g.ws_ctrl = 0;
     g.ws_flags = 256;
     g.ws_ring = g.ws_flags + ((static_cast<size_t>(g.chains) * 8 + 255) / 256) * 256;
@@ -1205,7 +1251,7 @@ cudaError_t forward(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)
     p.final_state = a.final_state;
     p.ctrl = reinterpret_cast<unsigned long long*>(ws + g.ws_ctrl);
     p.flags = reinterpret_cast<unsigned long long*>(ws + g.ws_flags);
-    p.epoch = ctx.epoch;
+    p.epoch = ctx.launch_tag(0);
     p.ring = reinterpret_cast<float*>(ws + g.ws_ring);
     p.status = ctx.status;
     p.wait_limit = ctx.wait_limit;
@@ -1225,6 +1271,8 @@ cudaError_t forward(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)
     p.seg_len = g.seg_len;
     p.nseg = g.nseg;
     p.items = g.items;
+    p.wrap = g.wrap;
+    p.grid = g.grid;
     p.skip_publish = g_skip_publish;
     return g.KH == 2 ? launch_kh<2>(tmX, tmB, tmC, tmY, p, g.grid, ctx.stream)
                      : launch_kh<1>(tmX, tmB, tmC, tmY, p, g.grid, ctx.stream);

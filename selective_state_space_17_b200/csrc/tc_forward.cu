@@ -1010,7 +1010,6 @@ cudaError_t launch(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)
     p.y = static_cast<__nv_bfloat16*>(a.y);
     p.final_state = a.final_state;
     p.flags = reinterpret_cast<unsigned long long*>(ws + w.flags);
-    p.epoch = ctx.epoch;
     p.ring = reinterpret_cast<float*>(ws + w.ring);
     p.seg_state = reinterpret_cast<float*>(ws + w.seg_state);
     p.seg_decay = reinterpret_cast<float*>(ws + w.seg_decay);
@@ -1033,9 +1032,11 @@ cudaError_t launch(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)
     cudaError_t e = cudaFuncSetAttribute(tc_forward_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
+    int nlaunch = 0;
     auto run = [&](int mode, int items) {
         p.mode = mode;
         p.items = items;
+        p.epoch = ctx.launch_tag(nlaunch++);
         const int grid = items < ctas_max ? items : ctas_max;
         tc_forward_kernel<<<grid, kThreads, smem, ctx.stream>>>(tmX, tmB, tmC, tmY, p);
         return cudaGetLastError();
