@@ -24,15 +24,16 @@
 //   mask    tril(S) as bf16 pairs, in place in TMEM (shared by the heads)
 //   X'      X'_h = diag(2^(c_h - cs_h,j) dt_h,j) X_h  (in place in shared memory)
 //   H'      H'_h = 2^(c_h) h_prev,h (bf16 operand), h <- 2^(c_h) h_prev,h in TMEM
-//   MMA3    Z   = C [H'_0 ... H'_KH-1]^T             (128 x 64 KH, K = N)
+//   Z init  Z_h,i = D_h x_h,i 2^(c_h - cs_h,i)          (the skip term over e_i)
+//   MMA3    Z  += C [H'_0 ... H'_KH-1]^T             (128 x 64 KH, K = N)
 //   MMA2    Z  += tril(S) [X'_0 ... X'_KH-1]         (128 x 64 KH, K = 128; A from TMEM)
 //   states  h  += B^T [X'_0 ... X'_KH-1]             (N x 64 KH, K = 128), so that
 //           h_new = 2^(cs_end - c) h (kept as a pending scalar)
-//   output  y_h,i = 2^(cs_h,i - c_h) Z_h,i + D_h x_h,i   (bf16, round to nearest even)
+//   output  y_h,i = e_h,i Z_h,i, e_h,i = 2^(cs_h,i - c_h)   (bf16, round to nearest even)
 //
 // A tile whose decay exceeds the bound ("exact form") keeps every factor <= 1:
 // X'_h = diag(2^(cs_end - cs_j) dt_j) X_h feeds the states only, H' = h_prev,
-// MMA3 writes C h_prev^T into Z, the output warps scale row i of Z by
+// Z starts from 0, MMA3 adds C h_prev^T, the output warps scale row i of Z by
 // 2^(cs_h,i) in place, and each head adds its own masked product
 // S~_h X_h with S~_h,ij = tril(S)_ij 2^(cs_h,i - cs_h,j) dt_h,j (built per head
 // in TMEM, X_h reloaded raw); then y = Z + D x. Both forms compute the chunked
@@ -40,31 +41,29 @@
 // inside a tile, the state across tiles (the composition of affine maps of
 // "Selective SSM guide" (auturnal.com), eq. (3)).
 //
-// Schedule. A chain is one batch row and one head group; it is cut into
-// segments of `seg_len` tiles, numbered segment-major, so a segment's
-// predecessor (the previous segment of its chain) is numbered `chains`
-// earlier. CTAs take segment numbers in order from a global ticket counter:
-// a CTA only waits on a segment that a running CTA took before it, so the
-// look-back cannot deadlock however many CTAs are resident. The state h of
-// the group's heads stays in TMEM from tile to tile; at a segment boundary it
+// Schedule. A chain is one batch row and one head group. The pieces a CTA runs
+// (see Pieces) come from a global ticket counter: each piece that starts
+// inside a chain waits only on a piece that a running CTA took before it, so
+// the look-back cannot deadlock however many CTAs are resident. The state h
+// of the group's heads stays in TMEM from tile to tile; between pieces it
 // travels through a per-chain slot in the workspace (release flag, bounded
 // acquire poll).
 //
-// Warp roles (416 threads), linked by full/empty mbarriers whose waits sleep
+// Warp roles (512 threads), linked by full/empty mbarriers whose waits sleep
 // and are bounded (no named barriers, so a role that gives up cannot leave
 // another stuck):
-//   warp 0        producer: segment tickets, TMA loads of C, B (2 stages) and X
-//                 (KH heads, 2 stages); TMEM allocation
+//   warp 0        producer: pieces, TMA loads of C, B (2 stages) and X (KH
+//                 heads, 2 stages); TMEM allocation
 //   warp 1        MMA stream A: MMA1 and states of each tile
 //   warp 2        MMA stream B: MMA3 and MMA2 (and the exact form's per-head
 //                 products, with the raw X reload)
-//   warps 3, 12   prologue, one head each: cumulative decay, tile record, X'
-//   warps 4-7     state and mask: h_prev -> H' and the scaled h, segment
+//   warp 3        prologue: cumulative decay of the tile's heads, tile record
+//   warps 4-7     state and mask: h_prev -> H' and the scaled h, piece
 //                 hand-off and final state; then S -> tril(S) (exact form:
 //                 S~_h per head)
-//   warps 8-11    output: y = e Z + D x written to global memory (x loaded
-//                 while the tile's products run); the exact form's row
-//                 scaling of Z
+//   warps 8-11    output: y = e Z stored from registers (exact form: the row
+//                 scaling of Z first, and y = Z + D x)
+//   warps 12-15   scale: X' in place and Z's initial value
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -87,18 +86,18 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kHardLog2 = 144.f;
 constexpr uint64_t kWaitNs = 2000000000ull;  // a role's wait on another gives up after ~2 s
 constexpr uint32_t kWaitPolls = 1u << 24;     // ... or after this many polls (each at most ~128 ns)
+constexpr uint32_t kRolePolls = 1u << 26;     // a role's wait on another: this many polls
 
-constexpr int kThreads = 416;
+constexpr int kThreads = 512;  // 16 warps of at most 128 registers: the whole register file
 constexpr int kWarpProducer = 0;
 constexpr int kWarpMmaA = 1;
 constexpr int kWarpMmaB = 2;
-constexpr int kWarpPro0 = 3;   // prologue of head 0
-constexpr int kWarpPro1 = 12;  // prologue of head 1
+constexpr int kWarpPro = 3;    // prologue of the tile's heads
 constexpr int kWgState = 4;    // warps 4..7
 constexpr int kWgOut = 8;      // warps 8..11
+constexpr int kWgScale = 12;   // warps 12..15
 constexpr int kSchedSlots = 4;
-constexpr int kPrefetch = 3;  // tiles ahead of the loads that the producer prefetches into L2
-constexpr int kSchedConsumers = 12;  // warps 1..12 read every ticket
+constexpr int kSchedConsumers = 15;  // warps 1..15 read every piece
 
 // TMEM columns (fp32, 128 lanes)
 constexpr uint32_t kColS = 0;    // 2 x 128: S, then tril(S) (bf16, cols 0-63) and S~_h (64-127)
@@ -113,8 +112,7 @@ struct Rec {
     float cref[2];    // reference value c of the scaled form
     float csend[2];   // cs of the tile's last token
     int hard;         // exact form for this tile
-    int hardh[2];     // per head, before the two are combined
-    int pad[9];
+    int pad[11];
 };
 static_assert(sizeof(Rec) == 1088, "record layout");
 
@@ -135,12 +133,12 @@ static_assert(Smem::kBytes <= 227 * 1024, "shared memory budget");
 
 enum Bar : int {
     kFullCB = 0,      // 2 (tx)
-    kEmptyCB = 2,     // 2 (states, MMA3)
+    kEmptyCB = 2,     // 2 (states, MMA3, the TMA store of y staged in C)
     kFullX = 4,       // 2 (tx)
-    kEmptyX = 6,      // 2 (states, MMA2, the TMA store of y)
-    kXpFull = 8,      // 2 (one per prologue warp)
-    kRecFull = 10,    // 2 (one per prologue warp)
-    kRecEmpty = 12,   // 2 (MMA B, four state and four output warps)
+    kEmptyX = 6,      // 2 (states, MMA2)
+    kXpFull = 8,      // 2 (four scale warps)
+    kRecFull = 10,    // 2 (the prologue warp)
+    kRecEmpty = 12,   // 2 (MMA B, four state, four output and four scale warps)
     kSFull = 14,      // 2
     kSFree = 16,      // 2
     kTrilFull = 18,   // 2 (four state warps)
@@ -149,7 +147,7 @@ enum Bar : int {
     kHpEmpty = 22,
     kStatesDone = 23,
     kZFull = 24,
-    kZEmpty = 25,     // four output warps
+    kZEmpty = 25,     // four output warps read Z
     kM3Done = 26,     // exact form
     kZScaled = 27,
     kRawX = 28,
@@ -159,22 +157,20 @@ enum Bar : int {
     kSchedEmpty = 35, // 4 (kSchedConsumers)
     kDrainA = 39,
     kDrainB = 40,
-    kHx = 41,         // the two prologue warps exchange their hard flags
+    kZInit = 41,      // four scale warps wrote Z's initial value
     kPub = 42,        // four state warps wrote a segment's end state
-    kYStaged = 43,    // four output warps wrote y over X'
-    kXRead = 44,      // 2: the states MMA of the tile in this X stage is done
+    kYStaged = 43,    // four output warps wrote y into the tile's C buffer
 };
 
-uint32_t bar_count(int i, int kh)
+uint32_t bar_count(int i)
 {
-    if (i == kEmptyCB || i == kEmptyCB + 1) return 2;
-    if (i == kEmptyX || i == kEmptyX + 1) return 3;
-    if (i == kRecFull || i == kRecFull + 1 || i == kHx) return kh;
-    if (i == kRecEmpty || i == kRecEmpty + 1) return 9;
+    if (i == kEmptyCB || i == kEmptyCB + 1) return 3;
+    if (i == kEmptyX || i == kEmptyX + 1) return 2;
+    if (i == kRecEmpty || i == kRecEmpty + 1) return 13;
     if (i == kTrilFull || i == kTrilFull + 1 || i == kZEmpty || i == kSlotFull || i == kHReady ||
-        i == kHpFull || i == kZScaled || i == kPub || i == kYStaged)
+        i == kHpFull || i == kZScaled || i == kPub || i == kXpFull || i == kXpFull + 1 || i == kZInit ||
+        i == kYStaged)
         return 4;
-    if (i == kXpFull || i == kXpFull + 1) return kh;
     if (i >= kSchedEmpty && i < kSchedEmpty + kSchedSlots) return kSchedConsumers;
     return 1;
 }
@@ -230,6 +226,7 @@ __device__ __forceinline__ bool wait_bounded_1(uint64_t* bar, uint32_t parity)
 {
     if (mbar_try_wait_short(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
+#pragma unroll 1
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait_short(bar, parity)) return true;
         if ((it & 63u) == 0u && (it >= kWaitPolls || global_timer_ns() - t0 > kWaitNs)) return false;
@@ -237,19 +234,19 @@ __device__ __forceinline__ bool wait_bounded_1(uint64_t* bar, uint32_t parity)
 }
 
 // Bounded wait of one thread on an mbarrier phase (each poll may suspend the
-// thread for a short time, so a hand-off wakes the waiter promptly; the clock
-// is read every 64 polls). A give-up puts the CTA into abort mode: later waits
-// return at once and every role runs out its loop; the status word reports it.
+// thread for up to ~128 ns, so a hand-off wakes the waiter promptly; it gives
+// up after kRolePolls polls, one to several seconds). A give-up puts the CTA
+// into abort mode: later waits return at once and every role runs out its
+// loop; the status word reports it.
+// (The bound is a poll count, so the loop inlined at every wait stays a few
+// instructions long.)
 __device__ __forceinline__ void wait_bar_1(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                            unsigned int* status)
 {
     if (*abort_flag) return;
-    if (mbar_try_wait_short(bar, parity)) return;
-    const uint64_t t0 = global_timer_ns();
-    for (uint32_t it = 1;; ++it) {
+#pragma unroll 1
+    for (uint32_t it = 0; it < kRolePolls; ++it)
         if (mbar_try_wait_short(bar, parity)) return;
-        if ((it & 63u) == 0u && (it >= kWaitPolls || global_timer_ns() - t0 > kWaitNs)) break;
-    }
     wait_gave_up(abort_flag, status);
 }
 
@@ -306,7 +303,7 @@ struct Pos {
 struct Pieces {
     long long u0 = 0, u1 = 0;
     int idx = 0;
-    __device__ int4 next(const GParams& p, volatile int* abort_flag)
+    __device__ __noinline__ int4 next(const GParams& p, volatile int* abort_flag)
     {
         const int4 none = make_int4(-1, 0, 0, 0);
         if (*abort_flag) return none;
@@ -349,7 +346,8 @@ struct SchedReader {
     // sequence after the bounded wait; in abort mode every reader ends at once
     // (the roles are linked by mbarriers only, so no role waits on a warp
     // that has left its loop for longer than a bounded wait).
-    __device__ int4 pop(uint8_t* sm, uint64_t* bars, volatile int* abort_flag, unsigned int* status)
+    __device__ __noinline__ int4 pop(uint8_t* sm, uint64_t* bars, volatile int* abort_flag,
+                                     unsigned int* status)
     {
         if (*abort_flag) return make_int4(-1, 0, 0, 0);  // aborted: every role just ends
         const uint32_t slot = n % kSchedSlots;
@@ -435,8 +433,6 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
 
     if (warp == kWarpProducer) {
         // ------------------------------------------------------------ producer
-        // Tickets are taken one segment ahead, so that the L2 prefetch of the
-        // tiles kPrefetch ahead runs across segment boundaries too.
         uint32_t npush = 0;
         Pieces src;
         auto fetch = [&]() {
@@ -469,45 +465,15 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             ++npush;
             return true;
         };
-        auto prefetch = [&](const Pos& q, int tile) {
-            const int t0 = tile * kT;
-            for (int h = 0; h < p.nkh; ++h) {
-                tma_prefetch_l2_4d(&tmC, h * 64, q.g, t0, q.b);
-                tma_prefetch_l2_4d(&tmB, h * 64, q.g, t0, q.b);
-            }
-#pragma unroll
-            for (int hh = 0; hh < KH; ++hh) tma_prefetch_l2_4d(&tmX, 0, q.hs0 + hh, t0, q.b);
-        };
-        const int4 kEnd = make_int4(-1, 0, 0, 0);
-        Pos s, nx;
+        Pos s;
         int4 pc = fetch();
         s.set(p, pc, KH);
         bool alive = push(pc);
-        pc = s.valid ? fetch() : kEnd;
-        nx.set(p, pc, KH);
-        int4 pc_nx = pc;
         int k = 0;
-        if (s.valid && elect_one_sync()) {
-            // the tiles before the prefetch distance
-            for (int d = 0; d < kPrefetch; ++d) {
-                if (s.tile + d < s.tile_end) prefetch(s, s.tile + d);
-                else if (nx.valid && nx.tile + (s.tile + d - s.tile_end) < nx.tile_end)
-                    prefetch(nx, nx.tile + (s.tile + d - s.tile_end));
-            }
-        }
-        __syncwarp();
         while (alive && s.valid && !*abort_flag) {
             const int st = k & 1;
             const uint32_t par = ((k >> 1) & 1) ^ 1;
             const int t0 = s.tile * kT;
-            // tile kPrefetch ahead into L2 (no shared memory, no completion)
-            if (kPrefetch > 0 && elect_one_sync()) {
-                const int ahead = s.tile + kPrefetch;
-                if (ahead < s.tile_end) prefetch(s, ahead);
-                else if (nx.valid && nx.tile + (ahead - s.tile_end) < nx.tile_end)
-                    prefetch(nx, nx.tile + (ahead - s.tile_end));
-            }
-            __syncwarp();
             wait_bar(bars + kEmptyCB + st, par, abort_flag, p.status);
             if (elect_one_sync()) {
                 mbar_arrive_expect_tx(bars + kFullCB + st, p.nkh * 2 * kHalf);
@@ -530,13 +496,12 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             __syncwarp();
             ++k;
             if (++s.tile >= s.tile_end) {
-                s = nx;
-                alive = push(pc_nx);
-                pc_nx = s.valid ? fetch() : kEnd;
-                nx.set(p, pc_nx, KH);
+                pc = fetch();
+                s.set(p, pc, KH);
+                alive = push(pc);
             }
         }
-        if (alive && s.valid) push(kEnd);  // aborted: tell every role to stop
+        if (alive && s.valid) push(make_int4(-1, 0, 0, 0));  // aborted: tell every role to stop
         // every load issued has landed before the CTA can exit
         for (int j = max(0, k - 2); j < k; ++j) {
             wait_bounded(bars + kFullCB + (j & 1), (j >> 1) & 1);
@@ -576,7 +541,6 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
                     mma_bf16(tmem + kColH, dbt0 + stage + q * (2048 >> 4), dx0 + stage + q * (2048 >> 4),
                              id_st, true);
                 mma_commit(bars + kStatesDone);
-                mma_commit(bars + kXRead + st);
                 mma_commit(bars + kEmptyCB + st);
                 mma_commit(bars + kEmptyX + st);
             }
@@ -605,12 +569,12 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             if (lane == 0) mbar_arrive(bars + kRecEmpty + st);
             wait_bar(bars + kFullCB + st, par, abort_flag, p.status);
             wait_bar(bars + kHpFull, k & 1, abort_flag, p.status);
-            wait_bar(bars + kZEmpty, (k & 1) ^ 1, abort_flag, p.status);
+            wait_bar(bars + kZInit, k & 1, abort_flag, p.status);  // Z holds D x / e (or 0)
             tc_fence_after_sync();
             if (elect_one_sync()) {
                 for (int q = 0; q < 4 * p.nkh; ++q)
                     mma_bf16(tmem + kColZ, dc0 + stage + (((q >> 2) * kHalf + (q & 3) * 32) >> 4),
-                             dhp + q * (2048 >> 4), id_y, q > 0);
+                             dhp + q * (2048 >> 4), id_y, true);
             }
             __syncwarp();
             if (!hard) {
@@ -678,97 +642,69 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
         if (elect_one_sync()) mma_commit(bars + kDrainB);
         __syncwarp();
         wait_bounded(bars + kDrainB, 0);
-    } else if (warp == kWarpPro0 || warp == kWarpPro1) {
-        // ------------------------------------ prologue: decay, record, X' (one head)
-        const int hh = warp == kWarpPro0 ? 0 : 1;
+    } else if (warp == kWarpPro) {
+        // ------------------------------ prologue: cumulative decay, tile record
         Walker<KH> w;
         w.begin(p, sm, bars, abort_flag);
-        if (hh < KH) {
-            // lane l holds tokens l, l + 32, l + 64, l + 96 of the tile
-            float dtv[4];
-            float Aval = 0.f;
-            auto fetch = [&](const Pos& q) {
-                const int rows = min(kT, p.L - q.tile * kT);
+        // lane l holds tokens l, l + 32, l + 64, l + 96 of the tile
+        float dtv[KH][4];
+        float Aval[KH];
+        auto fetch = [&](const Pos& q) {
+            const int rows = min(kT, p.L - q.tile * kT);
+#pragma unroll
+            for (int hh = 0; hh < KH; ++hh) {
                 const int hr = (q.hs0 + hh) / p.sub;
                 const size_t base = (static_cast<size_t>(q.b) * p.L + q.tile * kT) * p.Hr + hr;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int j = lane + 32 * u;
-                    dtv[u] = j < rows ? __ldg(p.dt + base + static_cast<size_t>(j) * p.Hr) : 0.f;
+                    dtv[hh][u] = j < rows ? __ldg(p.dt + base + static_cast<size_t>(j) * p.Hr) : 0.f;
                 }
-                Aval = __ldg(p.A + hr);
-            };
-            if (w.s.valid) fetch(w.s);
-            for (int k = 0; w.s.valid; ++k) {
-                const int st = k & 1;
-                const uint32_t par = (k >> 1) & 1;
-                const float dtc[4] = {dtv[0], dtv[1], dtv[2], dtv[3]};
-                const float Ah = Aval * kLog2e;
-                w.next(p, sm, bars, abort_flag);
-                if (w.s.valid) fetch(w.s);  // next tile's dt, in flight during this one
-
-                Rec& r = recs[st];
-                wait_bar(bars + kRecEmpty + st, par ^ 1, abort_flag, p.status);
-                float cs[4];
-                float carry = 0.f;
+                Aval[hh] = __ldg(p.A + hr);
+            }
+        };
+        if (w.s.valid) fetch(w.s);
+        for (int k = 0; w.s.valid; ++k) {
+            const int st = k & 1;
+            const uint32_t par = (k >> 1) & 1;
+            float dtc[KH][4], Ah[KH];
 #pragma unroll
+            for (int hh = 0; hh < KH; ++hh) {
+                Ah[hh] = Aval[hh] * kLog2e;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) dtc[hh][u] = dtv[hh][u];
+            }
+            w.next(p, sm, bars, abort_flag);
+            if (w.s.valid) fetch(w.s);  // next tile's dt, in flight during this one
+
+            Rec& rc = recs[st];
+            wait_bar(bars + kRecEmpty + st, par ^ 1, abort_flag, p.status);
+            int hard = 0;
+#pragma unroll
+            for (int hh = 0; hh < KH; ++hh) {
+                float carry = 0.f;
+#pragma unroll 1
                 for (int u = 0; u < 4; ++u) {
-                    float v = dtc[u] * Ah;
+                    // (the selects keep the 4 x KH values in registers)
+                    float v = (u == 0 ? dtc[hh][0] : u == 1 ? dtc[hh][1] : u == 2 ? dtc[hh][2] : dtc[hh][3]) * Ah[hh];
 #pragma unroll
                     for (int o = 1; o < 32; o <<= 1) {
                         const float t = __shfl_up_sync(0xffffffffu, v, o);
                         if (lane >= o) v += t;
                     }
-                    cs[u] = v + carry;
+                    rc.cs[hh][lane + 32 * u] = v + carry;
                     carry += __shfl_sync(0xffffffffu, v, 31);
                 }
-                const float cs_end = carry;
-#pragma unroll
-                for (int u = 0; u < 4; ++u) r.cs[hh][lane + 32 * u] = cs[u];
-                const int hard_h = -cs_end > kHardLog2 ? 1 : 0;
-                int hard = hard_h;
-                if (KH == 2) {
-                    if (lane == 0) {
-                        r.hardh[hh] = hard_h;
-                        mbar_arrive(bars + kHx);
-                    }
-                    wait_bar(bars + kHx, k & 1, abort_flag, p.status);
-                    hard = r.hardh[0] | r.hardh[1];
-                }
-                const float cref = 0.5f * cs_end;
+                // carry is the same in every lane: the tile's total decay
+                hard |= -carry > kHardLog2 ? 1 : 0;
                 if (lane == 0) {
-                    r.cref[hh] = cref;
-                    r.csend[hh] = cs_end;
-                    r.hard = hard;
+                    rc.cref[hh] = 0.5f * carry;
+                    rc.csend[hh] = carry;
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bars + kRecFull + st);
-
-                // X' = diag(f) X in place (fp32 product, one rounding). Chunk c of
-                // the head's tile (16 bytes) is in row c / 8 whatever the swizzle
-                // does inside the row; the factor of row j comes from lane j % 32.
-                float f[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    f[u] = ex2_approx(hard ? cs_end - cs[u] : cref - cs[u]) * dtc[u];
-                wait_bar(bars + kFullX + st, par, abort_flag, p.status);
-                uint4* xt = reinterpret_cast<uint4*>(sm + Smem::kX + st * 2 * kHalf + hh * kHalf);
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int c = j * 32 + lane;
-                    const float fr = __shfl_sync(0xffffffffu, f[j >> 3], (c >> 3) & 31);
-                    const uint4 v = xt[c];
-                    xt[c] = make_uint4(pack_bf16x2(fr * bf16_lo(v.x), fr * bf16_hi(v.x)),
-                                       pack_bf16x2(fr * bf16_lo(v.y), fr * bf16_hi(v.y)),
-                                       pack_bf16x2(fr * bf16_lo(v.z), fr * bf16_hi(v.z)),
-                                       pack_bf16x2(fr * bf16_lo(v.w), fr * bf16_hi(v.w)));
-                }
-                fence_async_shared();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bars + kXpFull + st);
             }
-        } else {
-            while (w.s.valid) w.next(p, sm, bars, abort_flag);  // KH = 1: read the tickets only
+            if (lane == 0) rc.hard = hard;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars + kRecFull + st);
         }
     } else if (warp >= kWgState && warp < kWgState + 4) {
         // ------------- state: H', the scaled h, segment hand-off; mask: tril(S)
@@ -781,7 +717,7 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
         w.begin(p, sm, bars, abort_flag);
         float s_pend[KH];  // true h = s_pend * (h in TMEM)
 #pragma unroll
-        for (int hh = 0; hh < KH; ++hh) s_pend[hh] = 1.f;
+        for (int hh = 0; hh < KH; ++hh) s_pend[hh] = 1.f;  // (indexed by constants only)
         Pos prev;
         prev.valid = false;
         bool prev_last = false;
@@ -841,18 +777,21 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             const int st = k & 1;
             const uint32_t par = (k >> 1) & 1;
             const Rec& rc = recs[st];
-            float sig3[KH], sigst[KH], snext[KH];
+            float f3[KH], ratio[KH], snext[KH];
             wait_bar(bars + kRecFull + st, par, abort_flag, p.status);
             const bool hard = rc.hard != 0;
+            const bool first = w.s.tile == w.s.tile_begin;
 #pragma unroll
             for (int hh = 0; hh < KH; ++hh) {
                 const float c = rc.cref[hh], ce = rc.csend[hh];
-                sig3[hh] = hard ? 1.f : ex2_approx(c);
-                sigst[hh] = ex2_approx(hard ? ce : c);
+                if (first) s_pend[hh] = 1.f;
+                // H' = 2^c s h (exact form: s h); the h the states MMA adds to is
+                // the same 2^c s h (exact form: 2^cs_end s h)
+                f3[hh] = (hard ? 1.f : ex2_approx(c)) * s_pend[hh];
+                ratio[hh] = hard ? ex2_approx(ce) : 1.f;
                 snext[hh] = hard ? 1.f : ex2_approx(ce - c);
             }
             // ---- H' (bf16 operand of MMA3) and the scaled state for tile k
-            const bool first = w.s.tile == w.s.tile_begin;
             if (first && w.s.seg > 0) {
                 // bounded acquire poll on the predecessor's flag, one per warp.
                 // Giving up only records the status: the call's results are
@@ -877,51 +816,69 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             }
             wait_bar(bars + kHpEmpty, (k & 1) ^ 1, abort_flag, p.status);
             tc_fence_after_sync();
+            if (first) {
+                // the piece's starting state goes into TMEM first: what the
+                // predecessor published (row r of [kN][kP]), the chain's initial
+                // state ([B][H][P][N]), or zero
+#pragma unroll 1
+                for (int j = 0; j < 4 * KH; ++j) {
+                    const int hh = j >> 2, q0 = (j & 3) * 16;
+                    uint32_t v[16];
+                    if (w.s.seg > 0) {
+                        const float4* src = reinterpret_cast<const float4*>(
+                            p.ring + ((static_cast<size_t>(w.s.chain) * KH + hh) * kN + r) * kP + q0);
 #pragma unroll
-            for (int hh = 0; hh < KH; ++hh) {
-                if (first) s_pend[hh] = 1.f;
-                const float f3 = sig3[hh] * s_pend[hh], fst = sigst[hh] * s_pend[hh];
-                const uint32_t a = tmem + lane_off + kColH + hh * 64;
-                uint32_t v[64];  // fp32 bits of row r of this head's h
-                if (!first) {
-                    tmem_ld64_sync(a, v);
-                } else if (w.s.seg > 0) {
-                    // what the predecessor published: row r of [kN][kP]
-                    const float4* src = reinterpret_cast<const float4*>(
-                        p.ring + ((static_cast<size_t>(w.s.chain) * KH + hh) * kN + r) * kP);
+                        for (int q = 0; q < 4; ++q) {
+                            const float4 u = __ldcg(src + q);
+                            v[4 * q] = __float_as_uint(u.x);
+                            v[4 * q + 1] = __float_as_uint(u.y);
+                            v[4 * q + 2] = __float_as_uint(u.z);
+                            v[4 * q + 3] = __float_as_uint(u.w);
+                        }
+                    } else if (p.init && n_live) {
+                        const float* src =
+                            p.init + (static_cast<size_t>(w.s.b) * p.Ht + w.s.hs0 + hh) * kP * Nst + q0 * Nst + r;
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const float4 u = __ldcg(src + q);
-                        v[4 * q] = __float_as_uint(u.x);
-                        v[4 * q + 1] = __float_as_uint(u.y);
-                        v[4 * q + 2] = __float_as_uint(u.z);
-                        v[4 * q + 3] = __float_as_uint(u.w);
+                        for (int q = 0; q < 16; ++q) v[q] = __float_as_uint(__ldg(src + q * Nst));
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) v[q] = 0u;
                     }
-                } else if (p.init && n_live) {
-                    // the chain's initial state, [B][H][P][N]
-                    const float* src = p.init + (static_cast<size_t>(w.s.b) * p.Ht + w.s.hs0 + hh) * kP * Nst + r;
-#pragma unroll
-                    for (int q = 0; q < 64; ++q) v[q] = __float_as_uint(__ldg(src + q * Nst));
-                } else {
-#pragma unroll
-                    for (int q = 0; q < 64; ++q) v[q] = 0u;
+                    tmem_st16(tmem + lane_off + kColH + hh * 64 + q0, v);
                 }
+                tmem_wait_st();
+            }
+            // 32 columns (a quarter of the heads' h) at a time: H' in shared
+            // memory, the scaled h back into TMEM
+#pragma unroll 1
+            for (int j = 0; j < 2 * KH; ++j) {
+                const int hh = j >> 1, half = j & 1;
+                const float fh = (KH == 2 && hh) ? f3[KH - 1] : f3[0];
+                const float rh = (KH == 2 && hh) ? ratio[KH - 1] : ratio[0];
+                const uint32_t a = tmem + lane_off + kColH + hh * 64 + half * 32;
+                uint32_t v[32];  // fp32 bits of columns 32 half .. 32 half + 31 of row r
+                tmem_ld32_sync(a, v);
+#pragma unroll
+                for (int q = 0; q < 32; ++q) v[q] = __float_as_uint(fh * __uint_as_float(v[q]));
                 uint8_t* row = sm + Smem::kHp + hh * kHalf + r * 128;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint32_t* u = v + c * 8;
-                    const uint4 hv = make_uint4(
-                        pack_bf16x2(f3 * __uint_as_float(u[0]), f3 * __uint_as_float(u[1])),
-                        pack_bf16x2(f3 * __uint_as_float(u[2]), f3 * __uint_as_float(u[3])),
-                        pack_bf16x2(f3 * __uint_as_float(u[4]), f3 * __uint_as_float(u[5])),
-                        pack_bf16x2(f3 * __uint_as_float(u[6]), f3 * __uint_as_float(u[7])));
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const int c = 4 * half + c4;
+                    const uint32_t* u = v + c4 * 8;
+                    const uint4 hv = make_uint4(pack_bf16x2(__uint_as_float(u[0]), __uint_as_float(u[1])),
+                                                pack_bf16x2(__uint_as_float(u[2]), __uint_as_float(u[3])),
+                                                pack_bf16x2(__uint_as_float(u[4]), __uint_as_float(u[5])),
+                                                pack_bf16x2(__uint_as_float(u[6]), __uint_as_float(u[7])));
                     *reinterpret_cast<uint4*>(row + (((c ^ r) & 7) << 4)) = hv;
                 }
+                if (hard) {
 #pragma unroll
-                for (int q = 0; q < 64; ++q) v[q] = __float_as_uint(fst * __uint_as_float(v[q]));
-                tmem_st64(a, v);
-                s_pend[hh] = snext[hh];
+                    for (int q = 0; q < 32; ++q) v[q] = __float_as_uint(rh * __uint_as_float(v[q]));
+                }
+                tmem_st32(a, v);
             }
+#pragma unroll
+            for (int hh = 0; hh < KH; ++hh) s_pend[hh] = snext[hh];
             tmem_wait_st();
             fence_async_shared();
             tc_fence_before_sync();
@@ -1017,15 +974,12 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             w.next(p, sm, bars, abort_flag);
         }
     } else if (warp >= kWgOut && warp < kWgOut + 4) {
-        // ------------------------------------------- output: y = e Z + D x.
-        // Thread r owns token row r of the tile and writes y_r over the row
-        // X'_r of the X stage, taking x_r for the D term back as X'_r / f_r (one
-        // more bf16 rounding of that term), or from global memory where f_r is
-        // too small for that (dt_r = 0, or an early token of an exact-form
-        // tile); one TMA store per head then writes the tile (rows past L are
-        // clipped), and the stage goes back to the producer once the stores
-        // have read it. Exact form: first Z_r *= 2^(cs_r), which the per-head
-        // masked products then add to.
+        // ------------------------------------------- output: y = e Z (+ D x).
+        // Thread r owns token row r of the tile. Scaled form: Z started from
+        // D x / e, so y = e Z. Exact form: Z_r *= 2^(cs_r) first, which the
+        // per-head masked products then add to, and y = Z + D x with x read
+        // from global memory. Each row of y (128 bytes per head) is stored
+        // from registers; rows past L are not written.
         const int wq = warp - kWgOut;
         const int r = wq * 32 + lane;  // token row i = TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
@@ -1036,24 +990,15 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             const Pos cur = w.s;
             const int st = k & 1;
             const uint32_t par = (k >> 1) & 1;
-            uint8_t* xs = sm + Smem::kX + st * 2 * kHalf;
             const bool live = r < p.L - cur.tile * kT;
-            float dtr[KH], Dh[KH];
-#pragma unroll
-            for (int hh = 0; hh < KH; ++hh) {
-                const int hr = (cur.hs0 + hh) / p.sub;
-                dtr[hh] = live ? __ldg(p.dt + (static_cast<size_t>(cur.b) * p.L + cur.tile * kT + r) * p.Hr + hr)
-                               : 0.f;
-                Dh[hh] = p.D ? __ldg(p.D + hr) : 0.f;
-            }
+            const size_t row0 = (static_cast<size_t>(cur.b) * p.L + cur.tile * kT + r) * p.Ht + cur.hs0;
             const Rec& rc = recs[st];
             wait_bar(bars + kRecFull + st, par, abort_flag, p.status);
             const bool hard = rc.hard != 0;
-            float f[KH], e[KH], zs[KH];
+            float e[KH], zs[KH];
 #pragma unroll
             for (int hh = 0; hh < KH; ++hh) {
                 const float ci = rc.cs[hh][r];
-                f[hh] = ex2_approx(hard ? rc.csend[hh] - ci : rc.cref[hh] - ci) * dtr[hh];
                 e[hh] = hard ? 1.f : ex2_approx(ci - rc.cref[hh]);
                 zs[hh] = ex2_approx(ci);
             }
@@ -1078,62 +1023,145 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
                 if (lane == 0) mbar_arrive(bars + kZScaled);
                 ++nh;
             }
-            // y over X' once MMA2 (Z full) and the states MMA (per-stage barrier)
-            // have read it
             wait_bar(bars + kZFull, k & 1, abort_flag, p.status);
-            wait_bar(bars + kXRead + st, par, abort_flag, p.status);
             tc_fence_after_sync();
+            // y into the tile's C buffer (dead since MMA3), 32 columns of Z at a
+            // time; Z is free for the next tile's initial value once the last
+            // columns are in registers
+            uint8_t* ys = sm + Smem::kC + st * 2 * kHalf + r * 128;
+            const bool add_dx = hard && p.D;
 #pragma unroll 1
-            for (int hh = 0; hh < KH; ++hh) {
-                uint8_t* row = xs + hh * kHalf + r * 128;
-                // per-head scalars by selection (no indexing by the loop counter)
-                const float fh = (KH == 2 && hh) ? f[KH - 1] : f[0];
-                const float Dhh = (KH == 2 && hh) ? Dh[KH - 1] : Dh[0];
+            for (int j = 0; j < 2 * KH; ++j) {
+                const int hh = j >> 1, half = j & 1;
+                uint32_t zv[32];
+                tmem_ld32_sync(tmem + lane_off + kColZ + hh * 64 + half * 32, zv);
+                if (j == 2 * KH - 1) {
+                    tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bars + kZEmpty);
+                }
                 const float eh = (KH == 2 && hh) ? e[KH - 1] : e[0];
-                // D x_r from X'_r / f_r, or from global memory where f_r is tiny
-                const bool from_xp = fh >= 0x1p-100f;
-                const float dx = from_xp ? Dhh / fh : Dhh;
-                const uint4* xg = reinterpret_cast<const uint4*>(
-                    p.x + ((static_cast<size_t>(cur.b) * p.L + cur.tile * kT + r) * p.Ht + cur.hs0 + hh) * kP);
-                uint32_t zv[64];
-                tmem_ld64_sync(tmem + lane_off + kColZ + hh * 64, zv);
+                float dh = 0.f;
+                if (add_dx) dh = __ldg(p.D + (cur.hs0 + hh) / p.sub);
+                const uint4* xg = reinterpret_cast<const uint4*>(p.x + (row0 + hh) * kP + half * 32);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint4* a = reinterpret_cast<uint4*>(row + (((c ^ r) & 7) << 4));
-                    uint4 xq = *a;
-                    if (!from_xp) xq = (live && Dhh != 0.f) ? __ldg(xg + c) : make_uint4(0u, 0u, 0u, 0u);
-                    const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    float xv[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) xv[u] = 0.f;
+                    if (add_dx && live) {
+                        // exact form: y = Z + D x, x from global memory
+                        const uint4 xq = __ldg(xg + c4);
+                        const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            xv[2 * u] = dh * bf16_lo(xw[u]);
+                            xv[2 * u + 1] = dh * bf16_hi(xw[u]);
+                        }
+                    }
                     uint32_t o[4];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
-                        const int j = c * 8 + u * 2;
-                        o[u] = pack_bf16x2(fmaf(eh, __uint_as_float(zv[j]), dx * bf16_lo(xw[u])),
-                                           fmaf(eh, __uint_as_float(zv[j + 1]), dx * bf16_hi(xw[u])));
+                        const int i = 8 * c4 + 2 * u;
+                        o[u] = pack_bf16x2(fmaf(eh, __uint_as_float(zv[i]), xv[2 * u]),
+                                           fmaf(eh, __uint_as_float(zv[i + 1]), xv[2 * u + 1]));
                     }
-                    *a = make_uint4(o[0], o[1], o[2], o[3]);
+                    const int c = 4 * half + c4;
+                    *reinterpret_cast<uint4*>(ys + hh * kHalf + (((c ^ r) & 7) << 4)) =
+                        make_uint4(o[0], o[1], o[2], o[3]);
                 }
             }
-            tc_fence_before_sync();
             fence_async_shared();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(bars + kZEmpty);
-                mbar_arrive(bars + kYStaged);
-            }
+            if (lane == 0) mbar_arrive(bars + kYStaged);
             if (r == 0) {
-                // one TMA store per head once all four warps staged their rows;
-                // the stage returns to the producer when the stores have read it
+                // one TMA store per head (rows past L are clipped); the C buffer
+                // goes back to the producer once the stores have read it
                 wait_bar_1(bars + kYStaged, k & 1, abort_flag, p.status);
 #pragma unroll
                 for (int hh = 0; hh < KH; ++hh)
-                    tma_store_4d(&tmY, xs + hh * kHalf, 0, cur.hs0 + hh, cur.tile * kT, cur.b);
+                    tma_store_4d(&tmY, ys + hh * kHalf, 0, cur.hs0 + hh, cur.tile * kT, cur.b);
                 tma_store_commit();
                 tma_store_wait_read();
-                mbar_arrive(bars + kEmptyX + st);
+                mbar_arrive(bars + kEmptyCB + st);
             }
             __syncwarp();
         }
         if (r == 0) tma_store_wait_all();
+    } else if (warp >= kWgScale) {
+        // ----------------------- scale: X' = diag(f) X, and Z's initial value.
+        // Thread r owns token row r: X'_r = f_r X_r in place (fp32 product, one
+        // rounding), f_r = 2^(c - cs_r) dt_r (exact form: 2^(cs_end - cs_r) dt_r);
+        // once the previous tile's Z has been read, Z_r starts from
+        // D x_r / e_r = D x_r 2^(c - cs_r) (exact form: 0), so that MMA3 and
+        // MMA2 accumulate onto the skip term.
+        const int wq = warp - kWgScale;
+        const int r = wq * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+        Walker<KH> w;
+        w.begin(p, sm, bars, abort_flag);
+        for (int k = 0; w.s.valid; ++k, w.next(p, sm, bars, abort_flag)) {
+            const Pos cur = w.s;
+            const int st = k & 1;
+            const uint32_t par = (k >> 1) & 1;
+            const bool live = r < p.L - cur.tile * kT;
+            float dtr[KH], Dh[KH];
+#pragma unroll
+            for (int hh = 0; hh < KH; ++hh) {
+                const int hr = (cur.hs0 + hh) / p.sub;
+                dtr[hh] = live ? __ldg(p.dt + (static_cast<size_t>(cur.b) * p.L + cur.tile * kT + r) * p.Hr + hr)
+                               : 0.f;
+                Dh[hh] = p.D ? __ldg(p.D + hr) : 0.f;
+            }
+            const Rec& rc = recs[st];
+            wait_bar(bars + kRecFull + st, par, abort_flag, p.status);
+            const bool hard = rc.hard != 0;
+            float f[KH], ie[KH];
+#pragma unroll
+            for (int hh = 0; hh < KH; ++hh) {
+                const float ci = rc.cs[hh][r];
+                f[hh] = ex2_approx(hard ? rc.csend[hh] - ci : rc.cref[hh] - ci) * dtr[hh];
+                ie[hh] = hard ? 0.f : Dh[hh] * ex2_approx(rc.cref[hh] - ci);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars + kRecEmpty + st);
+            // one pass over row r, 16 columns at a time: X' in place in shared
+            // memory, D x / e into Z (once the output warps have read the
+            // previous tile's Z)
+            wait_bar(bars + kZEmpty, (k & 1) ^ 1, abort_flag, p.status);
+            wait_bar(bars + kFullX + st, par, abort_flag, p.status);
+            tc_fence_after_sync();
+            uint8_t* xrow = sm + Smem::kX + st * 2 * kHalf + r * 128;
+#pragma unroll 1
+            for (int j = 0; j < 4 * KH; ++j) {
+                const int hh = j >> 2, c0 = 2 * (j & 3);
+                const float fr = (KH == 2 && hh) ? f[KH - 1] : f[0];
+                const float ih = (KH == 2 && hh) ? ie[KH - 1] : ie[0];
+                uint32_t zv[16];
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    uint4* a = reinterpret_cast<uint4*>(xrow + hh * kHalf + ((((c0 + h2) ^ r) & 7) << 4));
+                    const uint4 v = *a;
+                    const uint32_t xw[4] = {v.x, v.y, v.z, v.w};
+                    uint32_t o[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float x0 = bf16_lo(xw[u]), x1 = bf16_hi(xw[u]);
+                        o[u] = pack_bf16x2(fr * x0, fr * x1);
+                        zv[8 * h2 + 2 * u] = __float_as_uint(ih * x0);
+                        zv[8 * h2 + 2 * u + 1] = __float_as_uint(ih * x1);
+                    }
+                    *a = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+                tmem_st16(tmem + lane_off + kColZ + hh * 64 + c0 * 8, zv);
+            }
+            fence_async_shared();
+            tmem_wait_st();
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars + kXpFull + st);
+            if (lane == 0) mbar_arrive(bars + kZInit);
+        }
     }
 
     // ---- teardown
@@ -1255,7 +1283,7 @@ cudaError_t forward(const FwdArgs& a, void* workspace, const LaunchCtx& ctx)
     p.ring = reinterpret_cast<float*>(ws + g.ws_ring);
     p.status = ctx.status;
     p.wait_limit = ctx.wait_limit;
-    for (int i = 0; i < Smem::kNumBars; ++i) p.bar_counts[i] = bar_count(i, g.KH);
+    for (int i = 0; i < Smem::kNumBars; ++i) p.bar_counts[i] = bar_count(i);
     p.B = a.B;
     p.L = a.L;
     p.Ht = g.Ht;
