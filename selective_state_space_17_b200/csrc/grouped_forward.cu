@@ -54,9 +54,9 @@
 // another stuck):
 //   warp 0        producer: pieces, TMA loads of C, B (2 stages) and X (KH
 //                 heads, 2 stages); TMEM allocation
-//   warp 1        MMA stream A: MMA1 and states of each tile
-//   warp 2        MMA stream B: MMA3 and MMA2 (and the exact form's per-head
-//                 products, with the raw X reload)
+//   warp 1        MMA issue: MMA3, MMA2 (the exact form's per-head products,
+//                 with the raw X reload), MMA1 of the next tile, states
+//   warp 2        no role
 //   warp 3        prologue: cumulative decay of the tile's heads, tile record
 //   warps 4-7     state and mask: h_prev -> H' and the scaled h, piece
 //                 hand-off and final state; then S -> tril(S) (exact form:
@@ -90,14 +90,13 @@ constexpr uint32_t kRolePolls = 1u << 26;     // a role's wait on another: this 
 
 constexpr int kThreads = 512;  // 16 warps of at most 128 registers: the whole register file
 constexpr int kWarpProducer = 0;
-constexpr int kWarpMmaA = 1;
-constexpr int kWarpMmaB = 2;
+constexpr int kWarpMma = 1;
 constexpr int kWarpPro = 3;    // prologue of the tile's heads
 constexpr int kWgState = 4;    // warps 4..7
 constexpr int kWgOut = 8;      // warps 8..11
 constexpr int kWgScale = 12;   // warps 12..15
 constexpr int kSchedSlots = 4;
-constexpr int kSchedConsumers = 15;  // warps 1..15 read every piece
+constexpr int kSchedConsumers = 14;  // warps 1 and 3..15 read every piece
 
 // TMEM columns (fp32, 128 lanes)
 constexpr uint32_t kColS = 0;    // 2 x 128: S, then tril(S) (bf16, cols 0-63) and S~_h (64-127)
@@ -133,9 +132,9 @@ static_assert(Smem::kBytes <= 227 * 1024, "shared memory budget");
 
 enum Bar : int {
     kFullCB = 0,      // 2 (tx)
-    kEmptyCB = 2,     // 2 (states, MMA3, the TMA store of y staged in C)
+    kEmptyCB = 2,     // 2 (the MMAs of the tile, the TMA store of y staged in C)
     kFullX = 4,       // 2 (tx)
-    kEmptyX = 6,      // 2 (states, MMA2)
+    kEmptyX = 6,      // 2 (the MMAs of the tile)
     kXpFull = 8,      // 2 (four scale warps)
     kRecFull = 10,    // 2 (the prologue warp)
     kRecEmpty = 12,   // 2 (MMA B, four state, four output and four scale warps)
@@ -155,8 +154,7 @@ enum Bar : int {
     kSlotFree = 30,
     kSchedFull = 31,  // 4
     kSchedEmpty = 35, // 4 (kSchedConsumers)
-    kDrainA = 39,
-    kDrainB = 40,
+    kDrain = 39,
     kZInit = 41,      // four scale warps wrote Z's initial value
     kPub = 42,        // four state warps wrote a segment's end state
     kYStaged = 43,    // four output warps wrote y into the tile's C buffer
@@ -164,8 +162,8 @@ enum Bar : int {
 
 uint32_t bar_count(int i)
 {
-    if (i == kEmptyCB || i == kEmptyCB + 1) return 3;
-    if (i == kEmptyX || i == kEmptyX + 1) return 2;
+    if (i == kEmptyCB || i == kEmptyCB + 1) return 2;
+    if (i == kEmptyX || i == kEmptyX + 1) return 1;
     if (i == kRecEmpty || i == kRecEmpty + 1) return 13;
     if (i == kTrilFull || i == kTrilFull + 1 || i == kZEmpty || i == kSlotFull || i == kHReady ||
         i == kHpFull || i == kZScaled || i == kPub || i == kXpFull || i == kXpFull + 1 || i == kZInit ||
@@ -507,82 +505,65 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             wait_bounded(bars + kFullCB + (j & 1), (j >> 1) & 1);
             wait_bounded(bars + kFullX + (j & 1), (j >> 1) & 1);
         }
-    } else if (warp == kWarpMmaA) {
-        // ------------------------------------------------- stream A: MMA1, states
+    } else if (warp == kWarpMma) {
+        // ---------------------------------------------------------- MMA issue.
+        // One thread issues every product, per tile k in the order MMA3(k),
+        // MMA2(k), MMA1(k + 1), states(k): the products that make Z never
+        // queue behind the state update, and S of the next tile is ready when
+        // the state warps get to its mask.
         constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
         constexpr uint32_t id_st = idesc_bf16(128, 64 * KH, true, true);
+        constexpr uint32_t id_y = idesc_bf16(128, 64 * KH, false, true);
+        constexpr uint32_t id_y1 = idesc_bf16(128, 64, false, true);
         const uint64_t dc0 = sdesc_sw128(smem_addr(sm + Smem::kC), 16, 1024);
         const uint64_t db0 = sdesc_sw128(smem_addr(sm + Smem::kB), 16, 1024);
         const uint64_t dbt0 = sdesc_sw128(smem_addr(sm + Smem::kB), kHalf, 1024);  // B^T, MN-major
         const uint64_t dx0 = sdesc_sw128(smem_addr(sm + Smem::kX), kHalf, 1024);   // X', MN-major
-        Walker<KH> w;
-        w.begin(p, sm, bars, abort_flag);
-        for (int k = 0; w.s.valid; ++k, w.next(p, sm, bars, abort_flag)) {
-            const int st = k & 1;
-            const uint32_t par = (k >> 1) & 1;
-            const uint64_t stage = static_cast<uint64_t>(st * 2 * kHalf) >> 4;
-            wait_bar(bars + kFullCB + st, par, abort_flag, p.status);
-            wait_bar(bars + kSFree + st, par ^ 1, abort_flag, p.status);  // MMA2 of tile k - 2
+        const uint64_t dhp = sdesc_sw128(smem_addr(sm + Smem::kHp), kHalf, 1024);  // H', MN-major
+        auto stage_of = [](int kk) { return static_cast<uint64_t>((kk & 1) * 2 * kHalf) >> 4; };
+        // MMA1 of tile kk: S = C B^T into the S buffer of its stage
+        auto mma1 = [&](int kk) {
+            const int s1 = kk & 1;
+            const uint32_t p1 = (kk >> 1) & 1;
+            wait_bar(bars + kFullCB + s1, p1, abort_flag, p.status);
+            wait_bar(bars + kSFree + s1, p1 ^ 1, abort_flag, p.status);  // MMA2 of tile kk - 2
             tc_fence_after_sync();
             if (elect_one_sync()) {
                 for (int q = 0; q < 4 * p.nkh; ++q) {
                     const uint32_t off = ((q >> 2) * kHalf + (q & 3) * 32) >> 4;
-                    mma_bf16(tmem + kColS + st * 128, dc0 + stage + off, db0 + stage + off, id_s, q > 0);
+                    mma_bf16(tmem + kColS + s1 * 128, dc0 + stage_of(kk) + off, db0 + stage_of(kk) + off, id_s,
+                             q > 0);
                 }
-                mma_commit(bars + kSFull + st);
+                mma_commit(bars + kSFull + s1);
             }
             __syncwarp();
-            wait_bar(bars + kXpFull + st, par, abort_flag, p.status);
-            wait_bar(bars + kHReady, k & 1, abort_flag, p.status);
-            tc_fence_after_sync();
-            if (elect_one_sync()) {
-#pragma unroll
-                for (int q = 0; q < kT / 16; ++q)
-                    mma_bf16(tmem + kColH, dbt0 + stage + q * (2048 >> 4), dx0 + stage + q * (2048 >> 4),
-                             id_st, true);
-                mma_commit(bars + kStatesDone);
-                mma_commit(bars + kEmptyCB + st);
-                mma_commit(bars + kEmptyX + st);
-            }
-            __syncwarp();
-        }
-        if (elect_one_sync()) mma_commit(bars + kDrainA);
-        __syncwarp();
-        wait_bounded(bars + kDrainA, 0);
-    } else if (warp == kWarpMmaB) {
-        // -------------------------------------------------- stream B: MMA3, MMA2
-        constexpr uint32_t id_y = idesc_bf16(128, 64 * KH, false, true);
-        constexpr uint32_t id_y1 = idesc_bf16(128, 64, false, true);
-        const uint64_t dc0 = sdesc_sw128(smem_addr(sm + Smem::kC), 16, 1024);
-        const uint64_t dhp = sdesc_sw128(smem_addr(sm + Smem::kHp), kHalf, 1024);
-        const uint64_t dx0 = sdesc_sw128(smem_addr(sm + Smem::kX), kHalf, 1024);
+        };
         Walker<KH> w;
         w.begin(p, sm, bars, abort_flag);
         uint32_t nh = 0;  // exact-form tiles so far
-        for (int k = 0; w.s.valid; ++k, w.next(p, sm, bars, abort_flag)) {
+        if (w.s.valid) mma1(0);
+        for (int k = 0; w.s.valid; ++k) {
             const int st = k & 1;
             const uint32_t par = (k >> 1) & 1;
-            const uint64_t stage = static_cast<uint64_t>(st * 2 * kHalf) >> 4;
+            const uint64_t stage = stage_of(k);
             wait_bar(bars + kRecFull + st, par, abort_flag, p.status);
             const bool hard = recs[st].hard != 0;
+            const int tile_k = w.s.tile, hs0_k = w.s.hs0, b_k = w.s.b;
             __syncwarp();
             if (lane == 0) mbar_arrive(bars + kRecEmpty + st);
-            wait_bar(bars + kFullCB + st, par, abort_flag, p.status);
+            // ---- MMA3: Z += C H'^T (Z holds D x / e, or 0)
             wait_bar(bars + kHpFull, k & 1, abort_flag, p.status);
-            wait_bar(bars + kZInit, k & 1, abort_flag, p.status);  // Z holds D x / e (or 0)
+            wait_bar(bars + kZInit, k & 1, abort_flag, p.status);
             tc_fence_after_sync();
             if (elect_one_sync()) {
                 for (int q = 0; q < 4 * p.nkh; ++q)
                     mma_bf16(tmem + kColZ, dc0 + stage + (((q >> 2) * kHalf + (q & 3) * 32) >> 4),
                              dhp + q * (2048 >> 4), id_y, true);
+                if (!hard) mma_commit(bars + kHpEmpty);
             }
             __syncwarp();
             if (!hard) {
-                if (elect_one_sync()) {
-                    mma_commit(bars + kHpEmpty);
-                    mma_commit(bars + kEmptyCB + st);
-                }
-                __syncwarp();
+                // ---- MMA2: Z += tril(S) X'
                 wait_bar(bars + kTrilFull + st, par, abort_flag, p.status);
                 wait_bar(bars + kXpFull + st, par, abort_flag, p.status);
                 tc_fence_after_sync();
@@ -592,24 +573,20 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
                         mma_bf16_tmem_a(tmem + kColZ, tmem + kColS + st * 128 + q * 8,
                                         dx0 + stage + q * (2048 >> 4), id_y, true);
                     mma_commit(bars + kZFull);
-                    mma_commit(bars + kEmptyX + st);
                     mma_commit(bars + kSFree + st);
                 }
                 __syncwarp();
             } else {
                 // exact form: raw X into the H' buffer once MMA3 has read it,
                 // Z scaled by the output warps, then one masked product per head
-                if (elect_one_sync()) {
-                    mma_commit(bars + kEmptyCB + st);
-                    mma_commit(bars + kM3Done);
-                }
+                if (elect_one_sync()) mma_commit(bars + kM3Done);
                 __syncwarp();
                 wait_bar(bars + kM3Done, nh & 1, abort_flag, p.status);
                 if (elect_one_sync()) {
                     mbar_arrive_expect_tx(bars + kRawX, KH * kHalf);
 #pragma unroll
                     for (int hh = 0; hh < KH; ++hh)
-                        tma_load_4d(sm + Smem::kHp + hh * kHalf, &tmX, 0, w.s.hs0 + hh, w.s.tile * kT, w.s.b,
+                        tma_load_4d(sm + Smem::kHp + hh * kHalf, &tmX, 0, hs0_k + hh, tile_k * kT, b_k,
                                     bars + kRawX);
                 }
                 __syncwarp();
@@ -631,17 +608,32 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
                 }
                 if (elect_one_sync()) {
                     mma_commit(bars + kZFull);
-                    mma_commit(bars + kEmptyX + st);
                     mma_commit(bars + kSFree + st);
                     mma_commit(bars + kHpEmpty);
                 }
                 __syncwarp();
                 ++nh;
             }
+            // ---- MMA1 of the next tile, then the states of this one
+            w.next(p, sm, bars, abort_flag);
+            if (w.s.valid) mma1(k + 1);
+            wait_bar(bars + kXpFull + st, par, abort_flag, p.status);
+            wait_bar(bars + kHReady, k & 1, abort_flag, p.status);
+            tc_fence_after_sync();
+            if (elect_one_sync()) {
+#pragma unroll
+                for (int q = 0; q < kT / 16; ++q)
+                    mma_bf16(tmem + kColH, dbt0 + stage + q * (2048 >> 4), dx0 + stage + q * (2048 >> 4), id_st,
+                             true);
+                mma_commit(bars + kStatesDone);
+                mma_commit(bars + kEmptyCB + st);
+                mma_commit(bars + kEmptyX + st);
+            }
+            __syncwarp();
         }
-        if (elect_one_sync()) mma_commit(bars + kDrainB);
+        if (elect_one_sync()) mma_commit(bars + kDrain);
         __syncwarp();
-        wait_bounded(bars + kDrainB, 0);
+        wait_bounded(bars + kDrain, 0);
     } else if (warp == kWarpPro) {
         // ------------------------------ prologue: cumulative decay, tile record
         Walker<KH> w;
