@@ -541,8 +541,14 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
         Walker<KH> w;
         w.begin(p, sm, bars, abort_flag);
         uint32_t nh = 0;  // exact-form tiles so far
-        if (w.s.valid) mma1(0);
-        for (int k = 0; w.s.valid; ++k) {
+        // iteration k: the products of tile k (k >= 0), MMA1 of tile k + 1, the
+        // states of tile k (one MMA1 call site keeps the loop small)
+        for (int k = -1;; ++k) {
+            if (k < 0) {
+                if (!w.s.valid) break;
+                mma1(0);
+                continue;
+            }
             const int st = k & 1;
             const uint32_t par = (k >> 1) & 1;
             const uint64_t stage = stage_of(k);
@@ -568,7 +574,7 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
                 wait_bar(bars + kXpFull + st, par, abort_flag, p.status);
                 tc_fence_after_sync();
                 if (elect_one_sync()) {
-#pragma unroll
+#pragma unroll 1
                     for (int q = 0; q < kT / 16; ++q)
                         mma_bf16_tmem_a(tmem + kColZ, tmem + kColS + st * 128 + q * 8,
                                         dx0 + stage + q * (2048 >> 4), id_y, true);
@@ -616,12 +622,13 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             }
             // ---- MMA1 of the next tile, then the states of this one
             w.next(p, sm, bars, abort_flag);
-            if (w.s.valid) mma1(k + 1);
+            const bool more = w.s.valid;
+            if (more) mma1(k + 1);
             wait_bar(bars + kXpFull + st, par, abort_flag, p.status);
             wait_bar(bars + kHReady, k & 1, abort_flag, p.status);
             tc_fence_after_sync();
             if (elect_one_sync()) {
-#pragma unroll
+#pragma unroll 1
                 for (int q = 0; q < kT / 16; ++q)
                     mma_bf16(tmem + kColH, dbt0 + stage + q * (2048 >> 4), dx0 + stage + q * (2048 >> 4), id_st,
                              true);
@@ -630,6 +637,7 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
                 mma_commit(bars + kEmptyX + st);
             }
             __syncwarp();
+            if (!more) break;
         }
         if (elect_one_sync()) mma_commit(bars + kDrain);
         __syncwarp();
@@ -886,29 +894,23 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             wait_bar(bars + kSFull + st, par, abort_flag, p.status);
             tc_fence_after_sync();
             const uint32_t s_col = tmem + lane_off + kColS + st * 128;
-            // rows of lane quadrant wq need S blocks jb <= wq: blocks (0, 1) and
-            // (2, 3) are read as 64-column pairs, and each pair's bf16 output
-            // (32 columns at 32 jp) covers only columns read before
+            // 16 columns at a time: column block jc (fp32 columns 16 jc ..
+            // 16 jc + 15) becomes bf16 pairs in columns 8 jc .. 8 jc + 7, which
+            // were read before. Rows of lane quadrant wq keep j <= i, so only
+            // blocks jc <= 2 wq + 1 hold anything; the rest are zeros.
 #pragma unroll 1
-            for (int jp = 0; jp < 2; ++jp) {
-                uint32_t sv[64];
-                if (2 * jp <= wq) {
-                    tmem_ld64_sync(s_col + jp * 64, sv);
-                } else {
+            for (int jc = 0; jc < 8; ++jc) {
+                uint32_t sv[16];
+                if (jc <= 2 * wq + 1) tmem_ld16_sync(s_col + jc * 16, sv);
+                uint32_t pk[8];
 #pragma unroll
-                    for (int e = 0; e < 64; ++e) sv[e] = 0u;
+                for (int q = 0; q < 8; ++q) {
+                    const int j0 = jc * 16 + 2 * q;  // column of the pair's first value
+                    const float s0 = (jc <= 2 * wq + 1 && j0 <= r) ? __uint_as_float(sv[2 * q]) : 0.f;
+                    const float s1 = (jc <= 2 * wq + 1 && j0 + 1 <= r) ? __uint_as_float(sv[2 * q + 1]) : 0.f;
+                    pk[q] = pack_bf16x2(s0, s1);
                 }
-                // packed in place: word q takes values 2q, 2q + 1 (never behind q)
-#pragma unroll
-                for (int q = 0; q < 32; ++q) {
-                    const int e = 2 * q, jb = 2 * jp + (e >> 5), c = e & 31;
-                    // keep j <= i: blocks left of the diagonal whole, the
-                    // diagonal block up to column lane, nothing to the right
-                    const float s0 = (jb < wq || (jb == wq && c <= lane)) ? __uint_as_float(sv[e]) : 0.f;
-                    const float s1 = (jb < wq || (jb == wq && c + 1 <= lane)) ? __uint_as_float(sv[e + 1]) : 0.f;
-                    sv[q] = pack_bf16x2(s0, s1);
-                }
-                tmem_st32(s_col + jp * 32, sv);
+                tmem_st8(s_col + jc * 8, pk);
             }
             tmem_wait_st();
             tc_fence_before_sync();
@@ -935,11 +937,7 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
 #pragma unroll 1
                     for (int half = 0; half < 2; ++half) {
                         uint32_t wv[32];
-                        float tv[32];
-                        tmem_ld32(s_col + half * 32, tv);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) wv[e] = __float_as_uint(tv[e]);
+                        tmem_ld32_sync(s_col + half * 32, wv);
 #pragma unroll
                         for (int e = 0; e < 32; ++e) {
                             const int j0 = half * 64 + 2 * e;  // tokens j0, j0 + 1 (same 32-block)

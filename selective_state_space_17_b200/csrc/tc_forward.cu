@@ -602,8 +602,12 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 if (jb < wq) {
                     // block wholly left of the diagonal: row factor x column factor
                     float sv[32];
-                    tmem_ld32(s_col + jb * 32, sv);
-                    tmem_wait_ld();
+                    {
+                        uint32_t raw[32];
+                        tmem_ld32_sync(s_col + jb * 32, raw);
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) sv[q] = __uint_as_float(raw[q]);
+                    }
                     const float rf = ex2_approx(cs_i - r.cs[jb * 32 + 31]);
                     const float4* cf = reinterpret_cast<const float4*>(r.colf + jb * 32);
 #pragma unroll
@@ -618,8 +622,12 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     // position only selects values: rows diverge on j < i, and a
                     // per-element branch would serialise the warp.
                     float sv[32];
-                    tmem_ld32(s_col + jb * 32, sv);
-                    tmem_wait_ld();
+                    {
+                        uint32_t raw[32];
+                        tmem_ld32_sync(s_col + jb * 32, raw);
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) sv[q] = __uint_as_float(raw[q]);
+                    }
                     const float4* cs4 = reinterpret_cast<const float4*>(r.cs + jb * 32);
                     const float4* dt4 = reinterpret_cast<const float4*>(r.dt + jb * 32);
 #pragma unroll
@@ -750,8 +758,12 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 float sv[32];
-                tmem_ld32(tmem + lane_off + kColSt + sb * 64 + half * 32, sv);
-                tmem_wait_ld();
+                {
+                    uint32_t raw[32];
+                    tmem_ld32_sync(tmem + lane_off + kColSt + sb * 64 + half * 32, raw);
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) sv[q] = __uint_as_float(raw[q]);
+                }
 #pragma unroll
                 for (int q = 0; q < 32; ++q) h[half * 32 + q] = dec * h[half * 32 + q] + sv[q];
             }
@@ -809,9 +821,16 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
 #pragma unroll
                 for (int qd = 0; qd < 4; ++qd) {
                     float yd[16], ys[16];
-                    tmem_ld16(tmem + lane_off + kColY + sb * 64 + qd * 16, yd);
-                    tmem_ld16(tmem + lane_off + kColS + sb * 128 + 64 + qd * 16, ys);
-                    tmem_wait_ld();
+                    {
+                        uint32_t ra[16], rb[16];
+                        tmem_ld16x2_sync(tmem + lane_off + kColY + sb * 64 + qd * 16, ra,
+                                         tmem + lane_off + kColS + sb * 128 + 64 + qd * 16, rb);
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) {
+                            yd[q] = __uint_as_float(ra[q]);
+                            ys[q] = __uint_as_float(rb[q]);
+                        }
+                    }
 #pragma unroll
                     for (int h2 = 0; h2 < 2; ++h2) {
                         uint32_t o[4];
