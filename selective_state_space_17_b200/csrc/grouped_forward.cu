@@ -55,8 +55,8 @@
 //   warp 0        producer: pieces, TMA loads of C, B (2 stages) and X (KH
 //                 heads, 2 stages); TMEM allocation
 //   warp 1        MMA issue: MMA3, MMA2 (the exact form's per-head products,
-//                 with the raw X reload), MMA1 of the next tile, states
-//   warp 2        no role
+//                 with the raw X reload), MMA1 of the next tile
+//   warp 2        MMA issue: states
 //   warp 3        prologue: cumulative decay of the tile's heads, tile record
 //   warps 4-7     state and mask: h_prev -> H' and the scaled h, piece
 //                 hand-off and final state; then S -> tril(S) (exact form:
@@ -90,13 +90,14 @@ constexpr uint32_t kRolePolls = 1u << 26;     // a role's wait on another: this 
 
 constexpr int kThreads = 512;  // 16 warps of at most 128 registers: the whole register file
 constexpr int kWarpProducer = 0;
-constexpr int kWarpMma = 1;
+constexpr int kWarpMma = 1;    // MMA3, MMA2, MMA1
+constexpr int kWarpMmaS = 2;   // states
 constexpr int kWarpPro = 3;    // prologue of the tile's heads
 constexpr int kWgState = 4;    // warps 4..7
 constexpr int kWgOut = 8;      // warps 8..11
 constexpr int kWgScale = 12;   // warps 12..15
 constexpr int kSchedSlots = 4;
-constexpr int kSchedConsumers = 14;  // warps 1 and 3..15 read every piece
+constexpr int kSchedConsumers = 15;  // warps 1..15 read every piece
 
 // TMEM columns (fp32, 128 lanes)
 constexpr uint32_t kColS = 0;    // 2 x 128: S, then tril(S) (bf16, cols 0-63) and S~_h (64-127)
@@ -132,9 +133,9 @@ static_assert(Smem::kBytes <= 227 * 1024, "shared memory budget");
 
 enum Bar : int {
     kFullCB = 0,      // 2 (tx)
-    kEmptyCB = 2,     // 2 (the MMAs of the tile, the TMA store of y staged in C)
+    kEmptyCB = 2,     // 2 (the two MMA warps, the TMA store of y staged in C)
     kFullX = 4,       // 2 (tx)
-    kEmptyX = 6,      // 2 (the MMAs of the tile)
+    kEmptyX = 6,      // 2 (the two MMA warps)
     kXpFull = 8,      // 2 (four scale warps)
     kRecFull = 10,    // 2 (the prologue warp)
     kRecEmpty = 12,   // 2 (MMA B, four state, four output and four scale warps)
@@ -155,6 +156,7 @@ enum Bar : int {
     kSchedFull = 31,  // 4
     kSchedEmpty = 35, // 4 (kSchedConsumers)
     kDrain = 39,
+    kDrainS = 40,
     kZInit = 41,      // four scale warps wrote Z's initial value
     kPub = 42,        // four state warps wrote a segment's end state
     kYStaged = 43,    // four output warps wrote y into the tile's C buffer
@@ -162,8 +164,8 @@ enum Bar : int {
 
 uint32_t bar_count(int i)
 {
-    if (i == kEmptyCB || i == kEmptyCB + 1) return 2;
-    if (i == kEmptyX || i == kEmptyX + 1) return 1;
+    if (i == kEmptyCB || i == kEmptyCB + 1) return 3;
+    if (i == kEmptyX || i == kEmptyX + 1) return 2;
     if (i == kRecEmpty || i == kRecEmpty + 1) return 13;
     if (i == kTrilFull || i == kTrilFull + 1 || i == kZEmpty || i == kSlotFull || i == kHReady ||
         i == kHpFull || i == kZScaled || i == kPub || i == kXpFull || i == kXpFull + 1 || i == kZInit ||
@@ -506,18 +508,16 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             wait_bounded(bars + kFullX + (j & 1), (j >> 1) & 1);
         }
     } else if (warp == kWarpMma) {
-        // ---------------------------------------------------------- MMA issue.
-        // One thread issues every product, per tile k in the order MMA3(k),
-        // MMA2(k), MMA1(k + 1), states(k): the products that make Z never
-        // queue behind the state update, and S of the next tile is ready when
-        // the state warps get to its mask.
+        // ------------------------------------------------- MMA issue: Z and S.
+        // Per tile k: MMA3(k), MMA2(k), then MMA1(k + 1), so S of the next tile
+        // is ready when the state warps get to its mask. (An MMA issue blocks
+        // while the tensor pipe is busy, so the states products, which carry
+        // the recurrence from tile to tile, have their own issuing warp.)
         constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
-        constexpr uint32_t id_st = idesc_bf16(128, 64 * KH, true, true);
         constexpr uint32_t id_y = idesc_bf16(128, 64 * KH, false, true);
         constexpr uint32_t id_y1 = idesc_bf16(128, 64, false, true);
         const uint64_t dc0 = sdesc_sw128(smem_addr(sm + Smem::kC), 16, 1024);
         const uint64_t db0 = sdesc_sw128(smem_addr(sm + Smem::kB), 16, 1024);
-        const uint64_t dbt0 = sdesc_sw128(smem_addr(sm + Smem::kB), kHalf, 1024);  // B^T, MN-major
         const uint64_t dx0 = sdesc_sw128(smem_addr(sm + Smem::kX), kHalf, 1024);   // X', MN-major
         const uint64_t dhp = sdesc_sw128(smem_addr(sm + Smem::kHp), kHalf, 1024);  // H', MN-major
         auto stage_of = [](int kk) { return static_cast<uint64_t>((kk & 1) * 2 * kHalf) >> 4; };
@@ -620,10 +620,33 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
                 __syncwarp();
                 ++nh;
             }
-            // ---- MMA1 of the next tile, then the states of this one
+            if (elect_one_sync()) {
+                mma_commit(bars + kEmptyCB + st);
+                mma_commit(bars + kEmptyX + st);
+            }
+            __syncwarp();
+            // ---- MMA1 of the next tile
             w.next(p, sm, bars, abort_flag);
             const bool more = w.s.valid;
             if (more) mma1(k + 1);
+            if (!more) break;
+        }
+        if (elect_one_sync()) mma_commit(bars + kDrain);
+        __syncwarp();
+        wait_bounded(bars + kDrain, 0);
+    } else if (warp == kWarpMmaS) {
+        // --------------------------------------------- MMA issue: the states.
+        // h += B^T [X'_0 ... X'_KH-1] as soon as X' is in and the state warps
+        // have read and rescaled h.
+        constexpr uint32_t id_st = idesc_bf16(128, 64 * KH, true, true);
+        const uint64_t dbt0 = sdesc_sw128(smem_addr(sm + Smem::kB), kHalf, 1024);  // B^T, MN-major
+        const uint64_t dx0 = sdesc_sw128(smem_addr(sm + Smem::kX), kHalf, 1024);   // X', MN-major
+        Walker<KH> w;
+        w.begin(p, sm, bars, abort_flag);
+        for (int k = 0; w.s.valid; ++k, w.next(p, sm, bars, abort_flag)) {
+            const int st = k & 1;
+            const uint32_t par = (k >> 1) & 1;
+            const uint64_t stage = static_cast<uint64_t>(st * 2 * kHalf) >> 4;
             wait_bar(bars + kXpFull + st, par, abort_flag, p.status);
             wait_bar(bars + kHReady, k & 1, abort_flag, p.status);
             tc_fence_after_sync();
@@ -637,11 +660,10 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
                 mma_commit(bars + kEmptyX + st);
             }
             __syncwarp();
-            if (!more) break;
         }
-        if (elect_one_sync()) mma_commit(bars + kDrain);
+        if (elect_one_sync()) mma_commit(bars + kDrainS);
         __syncwarp();
-        wait_bounded(bars + kDrain, 0);
+        wait_bounded(bars + kDrainS, 0);
     } else if (warp == kWarpPro) {
         // ------------------------------ prologue: cumulative decay, tile record
         Walker<KH> w;
