@@ -86,7 +86,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kHardLog2 = 144.f;
 constexpr uint64_t kWaitNs = 2000000000ull;  // a role's wait on another gives up after ~2 s
 constexpr uint32_t kWaitPolls = 1u << 24;     // ... or after this many polls (each at most ~128 ns)
-constexpr uint32_t kRolePolls = 1u << 26;     // a role's wait on another: this many polls
+constexpr uint32_t kRolePolls = 1u << 22;     // a role's wait on another: this many polls (<= 1 us each)
 
 constexpr int kThreads = 512;  // 16 warps of at most 128 registers: the whole register file
 constexpr int kWarpProducer = 0;
@@ -233,20 +233,19 @@ __device__ __forceinline__ bool wait_bounded_1(uint64_t* bar, uint32_t parity)
     }
 }
 
-// Bounded wait of one thread on an mbarrier phase (each poll may suspend the
-// thread for up to ~128 ns, so a hand-off wakes the waiter promptly; it gives
-// up after kRolePolls polls, one to several seconds). A give-up puts the CTA
-// into abort mode: later waits return at once and every role runs out its
-// loop; the status word reports it.
-// (The bound is a poll count, so the loop inlined at every wait stays a few
-// instructions long.)
+// Bounded wait of one thread on an mbarrier phase: each poll suspends the
+// thread until the phase completes or ~1 us passes; it gives up after
+// kRolePolls polls (a fraction of a second to a few seconds). A give-up puts
+// the CTA into abort mode: later waits return at once and every role runs out
+// its loop; the status word reports it. (The bound is a poll count, so the
+// loop inlined at every wait stays a few instructions long.)
 __device__ __forceinline__ void wait_bar_1(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                            unsigned int* status)
 {
     if (*abort_flag) return;
 #pragma unroll 1
     for (uint32_t it = 0; it < kRolePolls; ++it)
-        if (mbar_try_wait_short(bar, parity)) return;
+        if (mbar_try_wait_1us(bar, parity)) return;
     wait_gave_up(abort_flag, status);
 }
 

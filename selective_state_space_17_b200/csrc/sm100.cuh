@@ -67,6 +67,22 @@ __device__ __forceinline__ bool mbar_try_wait_short(uint64_t* bar, uint32_t pari
     return ok != 0;
 }
 
+// The same with a 1 us suspend hint: a waiter that is woken by the phase
+// completing polls far less often (each poll is a shared-memory access that
+// the busy warps of the CTA would otherwise compete with).
+__device__ __forceinline__ bool mbar_try_wait_1us(uint64_t* bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(1000u)
+        : "memory");
+    return ok != 0;
+}
+
 // Non-blocking test of the phase of the given parity.
 __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity)
 {
