@@ -100,9 +100,9 @@ constexpr int kSchedSlots = 4;
 constexpr int kSchedConsumers = 15;  // warps 1..15 read every piece
 
 // TMEM columns (fp32, 128 lanes)
-constexpr uint32_t kColS = 0;    // 2 x 128: S, then tril(S) (bf16, cols 0-63) and S~_h (64-127)
-constexpr uint32_t kColH = 256;  // KH x 64: the states h, lane = state row n
-constexpr uint32_t kColZ = 384;  // KH x 64: Z, lane = token
+constexpr uint32_t kColS = 0;    // 128: S, then tril(S) (bf16, cols 0-63) and S~_h (64-127)
+constexpr uint32_t kColH = 128;  // KH x 64: the states h, lane = state row n
+constexpr uint32_t kColZ = 256;  // 2 x (KH x 64): Z of even and odd tiles, lane = token
 constexpr uint32_t kTmemCols = 512;
 
 constexpr uint32_t kHalf = 16384;  // one 128 x 64 bf16 block (a head's X, half of C or B)
@@ -139,15 +139,14 @@ enum Bar : int {
     kXpFull = 8,      // 2 (four scale warps)
     kRecFull = 10,    // 2 (the prologue warp)
     kRecEmpty = 12,   // 2 (MMA B, four state, four output and four scale warps)
-    kSFull = 14,      // 2
-    kSFree = 16,      // 2
+    kSFull = 14,      // MMA1 wrote S
+    kSFree = 16,      // MMA2 (exact form: the per-head products) read tril(S)
     kTrilFull = 18,   // 2 (four state warps)
     kHReady = 20,
     kHpFull = 21,
     kHpEmpty = 22,
     kStatesDone = 23,
-    kZFull = 24,
-    kZEmpty = 25,     // four output warps read Z
+    kZFull = 24,      // 2 (per Z buffer)
     kM3Done = 26,     // exact form
     kZScaled = 27,
     kRawX = 28,
@@ -157,9 +156,10 @@ enum Bar : int {
     kSchedEmpty = 35, // 4 (kSchedConsumers)
     kDrain = 39,
     kDrainS = 40,
-    kZInit = 41,      // four scale warps wrote Z's initial value
     kPub = 42,        // four state warps wrote a segment's end state
     kYStaged = 43,    // four output warps wrote y into the tile's C buffer
+    kZEmpty = 44,     // 2 (per Z buffer): four output warps read Z
+    kZInit = 46,      // 2 (per Z buffer): four scale warps wrote Z's initial value
 };
 
 uint32_t bar_count(int i)
@@ -167,8 +167,9 @@ uint32_t bar_count(int i)
     if (i == kEmptyCB || i == kEmptyCB + 1) return 3;
     if (i == kEmptyX || i == kEmptyX + 1) return 2;
     if (i == kRecEmpty || i == kRecEmpty + 1) return 13;
-    if (i == kTrilFull || i == kTrilFull + 1 || i == kZEmpty || i == kSlotFull || i == kHReady ||
-        i == kHpFull || i == kZScaled || i == kPub || i == kXpFull || i == kXpFull + 1 || i == kZInit ||
+    if (i == kTrilFull || i == kTrilFull + 1 || i == kZEmpty || i == kZEmpty + 1 || i == kSlotFull ||
+        i == kHReady || i == kHpFull || i == kZScaled || i == kPub || i == kXpFull || i == kXpFull + 1 ||
+        i == kZInit || i == kZInit + 1 ||
         i == kYStaged)
         return 4;
     if (i >= kSchedEmpty && i < kSchedEmpty + kSchedSlots) return kSchedConsumers;
@@ -525,15 +526,14 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             const int s1 = kk & 1;
             const uint32_t p1 = (kk >> 1) & 1;
             wait_bar(bars + kFullCB + s1, p1, abort_flag, p.status);
-            wait_bar(bars + kSFree + s1, p1 ^ 1, abort_flag, p.status);  // MMA2 of tile kk - 2
+            if (kk > 0) wait_bar(bars + kSFree, (kk - 1) & 1, abort_flag, p.status);  // MMA2 of tile kk - 1
             tc_fence_after_sync();
             if (elect_one_sync()) {
                 for (int q = 0; q < 4 * p.nkh; ++q) {
                     const uint32_t off = ((q >> 2) * kHalf + (q & 3) * 32) >> 4;
-                    mma_bf16(tmem + kColS + s1 * 128, dc0 + stage_of(kk) + off, db0 + stage_of(kk) + off, id_s,
-                             q > 0);
+                    mma_bf16(tmem + kColS, dc0 + stage_of(kk) + off, db0 + stage_of(kk) + off, id_s, q > 0);
                 }
-                mma_commit(bars + kSFull + s1);
+                mma_commit(bars + kSFull);
             }
             __syncwarp();
         };
@@ -558,11 +558,14 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             if (lane == 0) mbar_arrive(bars + kRecEmpty + st);
             // ---- MMA3: Z += C H'^T (Z holds D x / e, or 0)
             wait_bar(bars + kHpFull, k & 1, abort_flag, p.status);
-            wait_bar(bars + kZInit, k & 1, abort_flag, p.status);
+            const int zb = k & 1;
+            const uint32_t zpar = (k >> 1) & 1;
+            const uint32_t zcol = tmem + kColZ + zb * 128;
+            wait_bar(bars + kZInit + zb, zpar, abort_flag, p.status);
             tc_fence_after_sync();
             if (elect_one_sync()) {
                 for (int q = 0; q < 4 * p.nkh; ++q)
-                    mma_bf16(tmem + kColZ, dc0 + stage + (((q >> 2) * kHalf + (q & 3) * 32) >> 4),
+                    mma_bf16(zcol, dc0 + stage + (((q >> 2) * kHalf + (q & 3) * 32) >> 4),
                              dhp + q * (2048 >> 4), id_y, true);
                 if (!hard) mma_commit(bars + kHpEmpty);
             }
@@ -575,10 +578,9 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
                 if (elect_one_sync()) {
 #pragma unroll 1
                     for (int q = 0; q < kT / 16; ++q)
-                        mma_bf16_tmem_a(tmem + kColZ, tmem + kColS + st * 128 + q * 8,
-                                        dx0 + stage + q * (2048 >> 4), id_y, true);
-                    mma_commit(bars + kZFull);
-                    mma_commit(bars + kSFree + st);
+                        mma_bf16_tmem_a(zcol, tmem + kColS + q * 8, dx0 + stage + q * (2048 >> 4), id_y, true);
+                    mma_commit(bars + kZFull + zb);
+                    mma_commit(bars + kSFree);
                 }
                 __syncwarp();
             } else {
@@ -605,15 +607,15 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
                     if (elect_one_sync()) {
 #pragma unroll
                         for (int q = 0; q < kT / 16; ++q)
-                            mma_bf16_tmem_a(tmem + kColZ + hh * 64, tmem + kColS + st * 128 + 64 + q * 8,
+                            mma_bf16_tmem_a(zcol + hh * 64, tmem + kColS + 64 + q * 8,
                                             dhp + ((hh * kHalf) >> 4) + q * (2048 >> 4), id_y1, true);
                         mma_commit(bars + kSlotFree);
                     }
                     __syncwarp();
                 }
                 if (elect_one_sync()) {
-                    mma_commit(bars + kZFull);
-                    mma_commit(bars + kSFree + st);
+                    mma_commit(bars + kZFull + zb);
+                    mma_commit(bars + kSFree);
                     mma_commit(bars + kHpEmpty);
                 }
                 __syncwarp();
@@ -912,9 +914,9 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             // ---- mask of tile k: S -> tril(S), as bf16 pairs over the first 64
             // columns of the S buffer (block jb of 32 fp32 columns lands on
             // columns 16 jb .. 16 jb + 15, which are already read)
-            wait_bar(bars + kSFull + st, par, abort_flag, p.status);
+            wait_bar(bars + kSFull, k & 1, abort_flag, p.status);
             tc_fence_after_sync();
-            const uint32_t s_col = tmem + lane_off + kColS + st * 128;
+            const uint32_t s_col = tmem + lane_off + kColS;
             // 16 columns at a time: column block jc (fp32 columns 16 jc ..
             // 16 jc + 15) becomes bf16 pairs in columns 8 jc .. 8 jc + 7, which
             // were read before. Rows of lane quadrant wq keep j <= i, so only
@@ -1021,7 +1023,7 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
 #pragma unroll 1
                 for (int hh = 0; hh < KH; ++hh) {
                     uint32_t v[64];
-                    const uint32_t a = tmem + lane_off + kColZ + hh * 64;
+                    const uint32_t a = tmem + lane_off + kColZ + (k & 1) * 128 + hh * 64;
                     tmem_ld64_sync(a, v);
                     const float zsh = (KH == 2 && hh) ? zs[KH - 1] : zs[0];
 #pragma unroll
@@ -1034,22 +1036,22 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
                 if (lane == 0) mbar_arrive(bars + kZScaled);
                 ++nh;
             }
-            wait_bar(bars + kZFull, k & 1, abort_flag, p.status);
+            wait_bar(bars + kZFull + (k & 1), (k >> 1) & 1, abort_flag, p.status);
             tc_fence_after_sync();
             // y into the tile's C buffer (dead since MMA3), 32 columns of Z at a
-            // time; Z is free for the next tile's initial value once the last
-            // columns are in registers
+            // time; this Z buffer is free for the initial value of tile k + 2
+            // once the last columns are in registers
             uint8_t* ys = sm + Smem::kC + st * 2 * kHalf + r * 128;
             const bool add_dx = hard && p.D;
 #pragma unroll 1
             for (int j = 0; j < 2 * KH; ++j) {
                 const int hh = j >> 1, half = j & 1;
                 uint32_t zv[32];
-                tmem_ld32_sync(tmem + lane_off + kColZ + hh * 64 + half * 32, zv);
+                tmem_ld32_sync(tmem + lane_off + kColZ + (k & 1) * 128 + hh * 64 + half * 32, zv);
                 if (j == 2 * KH - 1) {
                     tc_fence_before_sync();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(bars + kZEmpty);
+                    if (lane == 0) mbar_arrive(bars + kZEmpty + (k & 1));
                 }
                 const float eh = (KH == 2 && hh) ? e[KH - 1] : e[0];
                 float dh = 0.f;
@@ -1103,7 +1105,7 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
         // ----------------------- scale: X' = diag(f) X, and Z's initial value.
         // Thread r owns token row r: X'_r = f_r X_r in place (fp32 product, one
         // rounding), f_r = 2^(c - cs_r) dt_r (exact form: 2^(cs_end - cs_r) dt_r);
-        // once the previous tile's Z has been read, Z_r starts from
+        // in the Z buffer the output warps have read for tile k - 2, Z_r starts from
         // D x_r / e_r = D x_r 2^(c - cs_r) (exact form: 0), so that MMA3 and
         // MMA2 accumulate onto the skip term.
         const int wq = warp - kWgScale;
@@ -1137,9 +1139,9 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             __syncwarp();
             if (lane == 0) mbar_arrive(bars + kRecEmpty + st);
             // one pass over row r, 16 columns at a time: X' in place in shared
-            // memory, D x / e into Z (once the output warps have read the
-            // previous tile's Z)
-            wait_bar(bars + kZEmpty, (k & 1) ^ 1, abort_flag, p.status);
+            // memory, D x / e into Z buffer k & 1 (once the output warps have
+            // read it for tile k - 2)
+            wait_bar(bars + kZEmpty + (k & 1), ((k >> 1) & 1) ^ 1, abort_flag, p.status);
             wait_bar(bars + kFullX + st, par, abort_flag, p.status);
             tc_fence_after_sync();
             uint8_t* xrow = sm + Smem::kX + st * 2 * kHalf + r * 128;
@@ -1164,14 +1166,14 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
                     }
                     *a = make_uint4(o[0], o[1], o[2], o[3]);
                 }
-                tmem_st16(tmem + lane_off + kColZ + hh * 64 + c0 * 8, zv);
+                tmem_st16(tmem + lane_off + kColZ + (k & 1) * 128 + hh * 64 + c0 * 8, zv);
             }
             fence_async_shared();
             tmem_wait_st();
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(bars + kXpFull + st);
-            if (lane == 0) mbar_arrive(bars + kZInit);
+            if (lane == 0) mbar_arrive(bars + kZInit + (k & 1));
         }
     }
 
