@@ -121,6 +121,12 @@ def code_digest(paths) -> str:
     return h.hexdigest()
 
 
+# The forward kernel that one ssd_forward call runs, by ssd_forward_path.
+KERNEL_OF_PATH = {1: "SIMT forward kernels", 2: "tc_forward_kernel",
+                  3: "tc_forward_kernel (segment-parallel) + segment_scan_kernel",
+                  4: "grouped_forward_kernel"}
+
+
 def recorded_traffic(workload: str):
     """DRAM bytes (read + write) of one launch from the ncu capture recorded in
     profiles/traffic.json, or None when the kernel's code (its sources without
@@ -500,6 +506,7 @@ def _report(args, w, rank, world, ms, per_step_ms, clk, inp, e2e_ms, host, ssd, 
     bound = "hbm" if t_hbm >= t_tc else "tensor"
     launches = ssd.kernel_count(w.B, w.L, w.H, w.P, w.G, w.N, w.chunk, code)
     traffic = recorded_traffic(w.name)
+    kernel = KERNEL_OF_PATH.get(ssd.forward_path(w.B, w.L, w.H, w.P, w.G, w.N, w.chunk, code), "?")
 
     result = None
     if rank == 0:
@@ -512,7 +519,8 @@ def _report(args, w, rank, world, ms, per_step_ms, clk, inp, e2e_ms, host, ssd, 
                        "heads": w.H, "headdim": w.P, "d_state": w.N, "groups": w.G,
                        "chunk": w.chunk, "parallelism": f"replicas x{world} (batch/head shards)",
                        "l2": "flushed between steps (256 MiB write, then 256 MiB read, outside the events)"},
-            "roofline": {"bound": bound, "achieved": achieved_gbs if bound == "hbm" else achieved_tflops,
+            "roofline": {"kernel": kernel, "bound": bound,
+                         "achieved": achieved_gbs if bound == "hbm" else achieved_tflops,
                          "peak": hbm_peak if bound == "hbm" else tc_peak,
                          "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
                          "frac": (achieved_gbs / hbm_peak) if bound == "hbm" else (achieved_tflops / tc_peak),
