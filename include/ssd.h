@@ -106,9 +106,14 @@ size_t ssd_workspace_size(int B, int L, int H, int P, int G, int N, int chunk, s
  *     2). Where a tile's total decay allows it, the decay mask is applied as
  *     a row and a column scaling around a reference point of the tile (the
  *     mask is a product of per-token decays); tiles of larger decay take an
- *     exact per-head form. Segments of a chain are handed to CTAs in order
- *     from a ticket counter, so a segment only waits on one that a running
- *     CTA already holds.
+ *     exact per-head form. The skip term D x enters as the initial value of
+ *     the accumulator (up to fp32 rounding the same sum). Work is handed to
+ *     CTAs through a ticket counter: with at least as many chains as SMs each
+ *     CTA takes one ticket (its rank) and an equal range of the chain-major
+ *     tile order, and the one piece it may wait on (the head of its first
+ *     chain) is run first by the CTA of the rank before, which took its ticket
+ *     earlier and so is running; with fewer chains, segments in ticket order.
+ *     No wait depends on a CTA that is not resident.
  *   - the per-head kernel takes the other sizes. With N > 128 it runs two
  *     passes over the state columns (n < 128, then the rest; each state column
  *     evolves on its own and y is a sum over columns): the first stores y with
