@@ -263,6 +263,27 @@ def test_step_matches_oracle(ssd, oracle, dtype):
     assert slice_rel_err(to_host_f64(state), str_, 1) < 1e-5
 
 
+@pytest.mark.parametrize("shape", [(41, 8, 64, 2, 128),   # 328 heads
+                                   (50, 6, 32, 3, 64),     # smaller state per head
+                                   (40, 8, 16, 1, 20)])    # N = 20: rows of 80 bytes
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_step_shapes(ssd, oracle, shape, dtype):
+    """More heads than one wave of CTAs, head counts that do not divide it,
+    smaller states and a state dim that is not a multiple of 32."""
+    B, H, P, G, N = shape
+    s = gen.make_step_inputs(B, H, P, G, N, dtype, seed=13)
+    io = (lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()) \
+        if dtype == "bf16" else (lambda a: torch.from_numpy(a).cuda())
+    state = torch.from_numpy(s.state).cuda()
+    y = ssd.step(io(s.x), torch.from_numpy(s.dt).cuda(), torch.from_numpy(s.A).cuda(),
+                 io(s.Bm), io(s.Cm), torch.from_numpy(s.D).cuda(), state)
+    ssd.poll_status()
+    f = lambda a: gen.to_f64(a, dtype)
+    yr, str_ = oracle.step(f(s.x), s.dt, s.A, f(s.Bm), f(s.Cm), s.D, s.state)
+    assert slice_rel_err(to_host_f64(y), yr, 1) < TOL[dtype]
+    assert slice_rel_err(to_host_f64(state), str_, 1) < 1e-5
+
+
 @pytest.mark.parametrize("N", [128, 13])
 def test_steps_reproduce_forward(ssd, N):
     inp = gen.make_inputs(2, 48, 4, 16, 2, N, "f32", seed=12)
