@@ -143,7 +143,13 @@ def forward(x, dt, A, Bm, Cm, D=None, chunk: int = 256, initial_state=None, y=No
             final_state=None, return_final_state: bool = True, workspace=None, stream=None):
     """SSD forward on CUDA tensors. x[B,L,H,P], dt[B,L,H] f32, A[H] f32,
     Bm/Cm[B,L,G,N], D[H] f32 or None, initial_state[B,H,P,N] f32 or None.
-    Returns (y, final_state) (final_state None if not requested)."""
+    Returns (y, final_state) (final_state None if not requested).
+
+    The call is asynchronous on `stream`. A device-side wait that gives up
+    (the per-head kernel's look-back when other work keeps some of its CTAs off
+    the SMs for seconds, or a test's fault injection) leaves y and final_state
+    undefined and records it in the stream's status word: poll_status() at a
+    synchronisation point raises SSDError then."""
     _need(x, "x")
     dev = x.device
     code = _dtype_code(x)
