@@ -215,6 +215,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// two fp32 products in one instruction, (a.x b.x, a.y b.y), each rounded to nearest
+__device__ __forceinline__ float2 mul2(float2 a, float2 b)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
 __device__ __noinline__ void wait_gave_up(volatile int* abort_flag, unsigned int* status)
 {
     record_status(status, kDevWaitTimeout);
@@ -918,22 +929,28 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             tc_fence_after_sync();
             const uint32_t s_col = tmem + lane_off + kColS;
             // 16 columns at a time: column block jc (fp32 columns 16 jc ..
-            // 16 jc + 15) becomes bf16 pairs in columns 8 jc .. 8 jc + 7, which
-            // were read before. Rows of lane quadrant wq keep j <= i, so only
-            // blocks jc <= 2 wq + 1 hold anything; the rest are zeros.
+            // 16 jc + 15) becomes bf16 pairs in columns 8 jc .. 8 jc + 7. Rows
+            // of lane quadrant wq (i = 32 wq + lane) keep j <= i: blocks left of
+            // 2 wq are packed whole, blocks 2 wq and 2 wq + 1 are cut at the
+            // diagonal, the rest become zeros. A block's output columns lie in
+            // a block read before it or in one this quadrant never reads.
+            const int jd = 2 * wq;
 #pragma unroll 1
-            for (int jc = 0; jc < 8; ++jc) {
+            for (int jc = 0; jc < jd + 2; ++jc) {
                 uint32_t sv[16];
-                if (jc <= 2 * wq + 1) tmem_ld16_sync(s_col + jc * 16, sv);
+                tmem_ld16_sync(s_col + jc * 16, sv);
+                const int lim = jc < jd ? 16 : r - jc * 16;  // keep column offsets <= lim
                 uint32_t pk[8];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const int j0 = jc * 16 + 2 * q;  // column of the pair's first value
-                    const float s0 = (jc <= 2 * wq + 1 && j0 <= r) ? __uint_as_float(sv[2 * q]) : 0.f;
-                    const float s1 = (jc <= 2 * wq + 1 && j0 + 1 <= r) ? __uint_as_float(sv[2 * q + 1]) : 0.f;
-                    pk[q] = pack_bf16x2(s0, s1);
-                }
+                for (int q = 0; q < 8; ++q)
+                    pk[q] = pack_bf16x2(2 * q <= lim ? __uint_as_float(sv[2 * q]) : 0.f,
+                                        2 * q + 1 <= lim ? __uint_as_float(sv[2 * q + 1]) : 0.f);
                 tmem_st8(s_col + jc * 8, pk);
+            }
+            {
+                const uint32_t z8[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll 1
+                for (int jc = jd + 2; jc < 8; ++jc) tmem_st8(s_col + jc * 8, z8);
             }
             tmem_wait_st();
             tc_fence_before_sync();
@@ -1043,45 +1060,74 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             // once the last columns are in registers
             uint8_t* ys = sm + Smem::kC + st * 2 * kHalf + r * 128;
             const bool add_dx = hard && p.D;
+            if (!add_dx) {
 #pragma unroll 1
-            for (int j = 0; j < 2 * KH; ++j) {
-                const int hh = j >> 1, half = j & 1;
-                uint32_t zv[32];
-                tmem_ld32_sync(tmem + lane_off + kColZ + (k & 1) * 128 + hh * 64 + half * 32, zv);
-                if (j == 2 * KH - 1) {
-                    tc_fence_before_sync();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bars + kZEmpty + (k & 1));
-                }
-                const float eh = (KH == 2 && hh) ? e[KH - 1] : e[0];
-                float dh = 0.f;
-                if (add_dx) dh = __ldg(p.D + (cur.hs0 + hh) / p.sub);
-                const uint4* xg = reinterpret_cast<const uint4*>(p.x + (row0 + hh) * kP + half * 32);
+                for (int j = 0; j < 2 * KH; ++j) {
+                    const int hh = j >> 1, half = j & 1;
+                    uint32_t zv[32];
+                    tmem_ld32_sync(tmem + lane_off + kColZ + (k & 1) * 128 + hh * 64 + half * 32, zv);
+                    if (j == 2 * KH - 1) {
+                        tc_fence_before_sync();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bars + kZEmpty + (k & 1));
+                    }
+                    const float eh = (KH == 2 && hh) ? e[KH - 1] : e[0];
 #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    float xv[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) xv[u] = 0.f;
-                    if (add_dx && live) {
-                        // exact form: y = Z + D x, x from global memory
-                        const uint4 xq = __ldg(xg + c4);
-                        const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        uint32_t o[4];
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
-                            xv[2 * u] = dh * bf16_lo(xw[u]);
-                            xv[2 * u + 1] = dh * bf16_hi(xw[u]);
+                            const int i = 8 * c4 + 2 * u;
+                            const float2 yv = mul2(make_float2(__uint_as_float(zv[i]), __uint_as_float(zv[i + 1])),
+                                                   make_float2(eh, eh));
+                            o[u] = pack_bf16x2(yv.x, yv.y);
                         }
+                        const int c = 4 * half + c4;
+                        *reinterpret_cast<uint4*>(ys + hh * kHalf + (((c ^ r) & 7) << 4)) =
+                            make_uint4(o[0], o[1], o[2], o[3]);
                     }
-                    uint32_t o[4];
+                }
+            } else {
+#pragma unroll 1
+                for (int j = 0; j < 2 * KH; ++j) {
+                    const int hh = j >> 1, half = j & 1;
+                    uint32_t zv[32];
+                    tmem_ld32_sync(tmem + lane_off + kColZ + (k & 1) * 128 + hh * 64 + half * 32, zv);
+                    if (j == 2 * KH - 1) {
+                        tc_fence_before_sync();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bars + kZEmpty + (k & 1));
+                    }
+                    const float eh = (KH == 2 && hh) ? e[KH - 1] : e[0];
+                    float dh = 0.f;
+                    if (add_dx) dh = __ldg(p.D + (cur.hs0 + hh) / p.sub);
+                    const uint4* xg = reinterpret_cast<const uint4*>(p.x + (row0 + hh) * kP + half * 32);
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int i = 8 * c4 + 2 * u;
-                        o[u] = pack_bf16x2(fmaf(eh, __uint_as_float(zv[i]), xv[2 * u]),
-                                           fmaf(eh, __uint_as_float(zv[i + 1]), xv[2 * u + 1]));
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        float xv[8];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) xv[u] = 0.f;
+                        if (add_dx && live) {
+                            // exact form: y = Z + D x, x from global memory
+                            const uint4 xq = __ldg(xg + c4);
+                            const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                xv[2 * u] = dh * bf16_lo(xw[u]);
+                                xv[2 * u + 1] = dh * bf16_hi(xw[u]);
+                            }
+                        }
+                        uint32_t o[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int i = 8 * c4 + 2 * u;
+                            o[u] = pack_bf16x2(fmaf(eh, __uint_as_float(zv[i]), xv[2 * u]),
+                                               fmaf(eh, __uint_as_float(zv[i + 1]), xv[2 * u + 1]));
+                        }
+                        const int c = 4 * half + c4;
+                        *reinterpret_cast<uint4*>(ys + hh * kHalf + (((c ^ r) & 7) << 4)) =
+                            make_uint4(o[0], o[1], o[2], o[3]);
                     }
-                    const int c = 4 * half + c4;
-                    *reinterpret_cast<uint4*>(ys + hh * kHalf + (((c ^ r) & 7) << 4)) =
-                        make_uint4(o[0], o[1], o[2], o[3]);
                 }
             }
             fence_async_shared();
@@ -1159,10 +1205,12 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
                     uint32_t o[4];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
-                        const float x0 = bf16_lo(xw[u]), x1 = bf16_hi(xw[u]);
-                        o[u] = pack_bf16x2(fr * x0, fr * x1);
-                        zv[8 * h2 + 2 * u] = __float_as_uint(ih * x0);
-                        zv[8 * h2 + 2 * u + 1] = __float_as_uint(ih * x1);
+                        const float2 xv = make_float2(bf16_lo(xw[u]), bf16_hi(xw[u]));
+                        const float2 xs = mul2(xv, make_float2(fr, fr));
+                        const float2 zs = mul2(xv, make_float2(ih, ih));
+                        o[u] = pack_bf16x2(xs.x, xs.y);
+                        zv[8 * h2 + 2 * u] = __float_as_uint(zs.x);
+                        zv[8 * h2 + 2 * u + 1] = __float_as_uint(zs.y);
                     }
                     *a = make_uint4(o[0], o[1], o[2], o[3]);
                 }
