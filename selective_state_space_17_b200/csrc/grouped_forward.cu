@@ -215,6 +215,19 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// a read-only load issued where it stands (not moved towards its first use)
+__device__ __forceinline__ float ldg_f32_now(const float* ptr)
+{
+    float v;
+    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(ptr));
+    return v;
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* ptr)
+{
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
+}
+
 // two fp32 products in one instruction, (a.x b.x, a.y b.y), each rounded to nearest
 __device__ __forceinline__ float2 mul2(float2 a, float2 b)
 {
@@ -680,7 +693,7 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
         // ------------------------------ prologue: cumulative decay, tile record
         Walker<KH> w;
         w.begin(p, sm, bars, abort_flag);
-        // lane l holds tokens l, l + 32, l + 64, l + 96 of the tile
+        // lane l holds tokens 4 l .. 4 l + 3 of the tile
         float dtv[KH][4];
         float Aval[KH];
         auto fetch = [&](const Pos& q) {
@@ -691,10 +704,21 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
                 const size_t base = (static_cast<size_t>(q.b) * p.L + q.tile * kT) * p.Hr + hr;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const int j = lane + 32 * u;
-                    dtv[hh][u] = j < rows ? __ldg(p.dt + base + static_cast<size_t>(j) * p.Hr) : 0.f;
+                    const int j = 4 * lane + u;
+                    dtv[hh][u] = j < rows ? ldg_f32_now(p.dt + base + static_cast<size_t>(j) * p.Hr) : 0.f;
                 }
                 Aval[hh] = __ldg(p.A + hr);
+            }
+            // the dt lines of the tiles two and three ahead into L2
+#pragma unroll
+            for (int ahead = 2; ahead <= 3; ++ahead) {
+                const int t = (q.tile + ahead) * kT;
+                const int hr = q.hs0 / p.sub;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int j = t + lane + 32 * u;
+                    if (j < p.L) prefetch_l2(p.dt + (static_cast<size_t>(q.b) * p.L + j) * p.Hr + hr);
+                }
             }
         };
         if (w.s.valid) fetch(w.s);
@@ -716,24 +740,28 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             int hard = 0;
 #pragma unroll
             for (int hh = 0; hh < KH; ++hh) {
-                float carry = 0.f;
-#pragma unroll 1
-                for (int u = 0; u < 4; ++u) {
-                    // (the selects keep the 4 x KH values in registers)
-                    float v = (u == 0 ? dtc[hh][0] : u == 1 ? dtc[hh][1] : u == 2 ? dtc[hh][2] : dtc[hh][3]) * Ah[hh];
+                // running sum over the lane's four tokens, then one scan over
+                // the lanes' totals
+                float a[4];
+                a[0] = dtc[hh][0] * Ah[hh];
 #pragma unroll
-                    for (int o = 1; o < 32; o <<= 1) {
-                        const float t = __shfl_up_sync(0xffffffffu, v, o);
-                        if (lane >= o) v += t;
-                    }
-                    rc.cs[hh][lane + 32 * u] = v + carry;
-                    carry += __shfl_sync(0xffffffffu, v, 31);
+                for (int u = 1; u < 4; ++u) a[u] = fmaf(dtc[hh][u], Ah[hh], a[u - 1]);
+                float incl = a[3];
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float t = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += t;
                 }
-                // carry is the same in every lane: the tile's total decay
-                hard |= -carry > kHardLog2 ? 1 : 0;
+                float excl = __shfl_up_sync(0xffffffffu, incl, 1);
+                if (lane == 0) excl = 0.f;
+                const float total = __shfl_sync(0xffffffffu, incl, 31);
+                *reinterpret_cast<float4*>(&rc.cs[hh][4 * lane]) =
+                    make_float4(excl + a[0], excl + a[1], excl + a[2], excl + a[3]);
+                // total is the same in every lane: the tile's total decay
+                hard |= -total > kHardLog2 ? 1 : 0;
                 if (lane == 0) {
-                    rc.cref[hh] = 0.5f * carry;
-                    rc.csend[hh] = carry;
+                    rc.cref[hh] = 0.5f * total;
+                    rc.csend[hh] = total;
                 }
             }
             if (lane == 0) rc.hard = hard;
