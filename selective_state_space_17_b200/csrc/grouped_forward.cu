@@ -403,6 +403,137 @@ struct Walker {
     }
 };
 
+// Exact-form tiles are rare; their parts of the role loops live out of line so
+// that the hot loops stay compact in the instruction cache.
+
+// State warps: S~_h,ij = tril(S)_ij 2^(cs_i - cs_j) dt_j of each head into
+// columns 64-127 of the S buffer, handed to the MMA warp one head at a time.
+template <int KH>
+__device__ __noinline__ void state_exact_stilde(const GParams& p, uint64_t* bars, volatile int* abort_flag,
+                                                const Rec& rc, int b, int tile, int hs0, uint32_t s_col,
+                                                uint32_t nh, int r, int lane)
+{
+    const int rows = min(kT, p.L - tile * kT);
+#pragma unroll
+    for (int hh = 0; hh < KH; ++hh) {
+        const int hr = (hs0 + hh) / p.sub;
+        const size_t base = (static_cast<size_t>(b) * p.L + tile * kT) * p.Hr + hr;
+        float dtl[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = lane + 32 * u;
+            dtl[u] = j < rows ? __ldg(p.dt + base + static_cast<size_t>(j) * p.Hr) : 0.f;
+        }
+        const float cs_i = rc.cs[hh][r];
+        const uint32_t u_slot = nh * KH + hh;
+        wait_bar(bars + kSlotFree, (u_slot & 1) ^ 1, abort_flag, p.status);
+        tc_fence_after_sync();
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+            uint32_t wv[32];
+            tmem_ld32_sync(s_col + half * 32, wv);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int j0 = half * 64 + 2 * e;  // tokens j0, j0 + 1 (same 32-block)
+                const float dsrc = half ? dtl[2 + (e >> 4)] : dtl[e >> 4];
+                const float d0 = __shfl_sync(0xffffffffu, dsrc, j0 & 31);
+                const float d1 = __shfl_sync(0xffffffffu, dsrc, (j0 + 1) & 31);
+                const float m0 = ex2_approx(fminf(cs_i - rc.cs[hh][j0], 0.f)) * d0;
+                const float m1 = ex2_approx(fminf(cs_i - rc.cs[hh][j0 + 1], 0.f)) * d1;
+                wv[e] = pack_bf16x2(bf16_lo(wv[e]) * m0, bf16_hi(wv[e]) * m1);
+            }
+            tmem_st32(s_col + 64 + half * 32, wv);
+        }
+        tmem_wait_st();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars + kSlotFull);
+    }
+}
+
+// State warps, exact form: row r of each head's h in TMEM times rh.
+template <int KH>
+__device__ __noinline__ void state_exact_rescale(uint32_t hcol, float r0, float r1)
+{
+#pragma unroll 1
+    for (int hh = 0; hh < KH; ++hh) {
+        uint32_t v[64];
+        tmem_ld64_sync(hcol + hh * 64, v);
+        const float rh = hh ? r1 : r0;
+#pragma unroll
+        for (int q = 0; q < 64; ++q) v[q] = __float_as_uint(rh * __uint_as_float(v[q]));
+        tmem_st64(hcol + hh * 64, v);
+    }
+}
+
+// Output warps, exact form: Z_r *= 2^(cs_r) once MMA3 is done, before the
+// per-head masked products add to it.
+template <int KH>
+__device__ __noinline__ void out_exact_scale(uint64_t* bars, volatile int* abort_flag, unsigned int* status,
+                                             uint32_t zaddr, float zs0, float zs1, uint32_t nh, int lane)
+{
+    wait_bar(bars + kM3Done, nh & 1, abort_flag, status);
+    tc_fence_after_sync();
+#pragma unroll 1
+    for (int hh = 0; hh < KH; ++hh) {
+        uint32_t v[64];
+        const uint32_t a = zaddr + hh * 64;
+        tmem_ld64_sync(a, v);
+        const float zsh = hh ? zs1 : zs0;
+#pragma unroll
+        for (int q = 0; q < 64; ++q) v[q] = __float_as_uint(__uint_as_float(v[q]) * zsh);
+        tmem_st64(a, v);
+    }
+    tmem_wait_st();
+    tc_fence_before_sync();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bars + kZScaled);
+}
+
+// Output warps, exact form with a skip term: y = Z + D x, x from global memory.
+template <int KH>
+__device__ __noinline__ void out_exact_epilogue(uint64_t* bars, uint32_t zaddr, uint8_t* ys,
+                                                const __nv_bfloat16* x, size_t row0, const float* D, int hs0,
+                                                int sub, bool live, int r, int lane, int zb)
+{
+#pragma unroll 1
+    for (int j = 0; j < 2 * KH; ++j) {
+        const int hh = j >> 1, half = j & 1;
+        uint32_t zv[32];
+        tmem_ld32_sync(zaddr + hh * 64 + half * 32, zv);
+        if (j == 2 * KH - 1) {
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars + kZEmpty + zb);
+        }
+        const float dh = __ldg(D + (hs0 + hh) / sub);
+        const uint4* xg = reinterpret_cast<const uint4*>(x + (row0 + hh) * kP + half * 32);
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+            float xv[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) xv[u] = 0.f;
+            if (live) {
+                const uint4 xq = __ldg(xg + c4);
+                const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    xv[2 * u] = dh * bf16_lo(xw[u]);
+                    xv[2 * u + 1] = dh * bf16_hi(xw[u]);
+                }
+            }
+            uint32_t o[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = 8 * c4 + 2 * u;
+                o[u] = pack_bf16x2(__uint_as_float(zv[i]) + xv[2 * u], __uint_as_float(zv[i + 1]) + xv[2 * u + 1]);
+            }
+            const int c = 4 * half + c4;
+            *reinterpret_cast<uint4*>(ys + hh * kHalf + (((c ^ r) & 7) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    }
+}
+
 template <int KH>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
@@ -594,7 +725,7 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
                 if (!hard) mma_commit(bars + kHpEmpty);
             }
             __syncwarp();
-            if (!hard) {
+            if (__builtin_expect(!hard, 1)) {
                 // ---- MMA2: Z += tril(S) X'
                 wait_bar(bars + kTrilFull + st, par, abort_flag, p.status);
                 wait_bar(bars + kXpFull + st, par, abort_flag, p.status);
@@ -916,7 +1047,6 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             for (int j = 0; j < 2 * KH; ++j) {
                 const int hh = j >> 1, half = j & 1;
                 const float fh = (KH == 2 && hh) ? f3[KH - 1] : f3[0];
-                const float rh = (KH == 2 && hh) ? ratio[KH - 1] : ratio[0];
                 const uint32_t a = tmem + lane_off + kColH + hh * 64 + half * 32;
                 uint32_t v[32];  // fp32 bits of columns 32 half .. 32 half + 31 of row r
                 tmem_ld32_sync(a, v);
@@ -933,11 +1063,12 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
                                                 pack_bf16x2(__uint_as_float(u[6]), __uint_as_float(u[7])));
                     *reinterpret_cast<uint4*>(row + (((c ^ r) & 7) << 4)) = hv;
                 }
-                if (hard) {
-#pragma unroll
-                    for (int q = 0; q < 32; ++q) v[q] = __float_as_uint(rh * __uint_as_float(v[q]));
-                }
                 tmem_st32(a, v);
+            }
+            // exact form: the h the states MMA adds to is 2^cs_end s h
+            if (__builtin_expect(hard, 0)) {
+                tmem_wait_st();
+                state_exact_rescale<KH>(tmem + lane_off + kColH, ratio[0], ratio[KH - 1]);
             }
 #pragma unroll
             for (int hh = 0; hh < KH; ++hh) s_pend[hh] = snext[hh];
@@ -984,45 +1115,10 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(bars + kTrilFull + st);
-            if (hard) {
+            if (__builtin_expect(hard, 0)) {
                 // exact form: S~_h,ij = tril(S)_ij 2^(cs_i - cs_j) dt_j into
                 // columns 64-127, one head at a time
-                const int rows = min(kT, p.L - w.s.tile * kT);
-#pragma unroll
-                for (int hh = 0; hh < KH; ++hh) {
-                    const int hr = (w.s.hs0 + hh) / p.sub;
-                    const size_t base = (static_cast<size_t>(w.s.b) * p.L + w.s.tile * kT) * p.Hr + hr;
-                    float dtl[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int j = lane + 32 * u;
-                        dtl[u] = j < rows ? __ldg(p.dt + base + static_cast<size_t>(j) * p.Hr) : 0.f;
-                    }
-                    const float cs_i = rc.cs[hh][r];
-                    const uint32_t u_slot = nh * KH + hh;
-                    wait_bar(bars + kSlotFree, (u_slot & 1) ^ 1, abort_flag, p.status);
-                    tc_fence_after_sync();
-#pragma unroll 1
-                    for (int half = 0; half < 2; ++half) {
-                        uint32_t wv[32];
-                        tmem_ld32_sync(s_col + half * 32, wv);
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const int j0 = half * 64 + 2 * e;  // tokens j0, j0 + 1 (same 32-block)
-                            const float dsrc = half ? dtl[2 + (e >> 4)] : dtl[e >> 4];
-                            const float d0 = __shfl_sync(0xffffffffu, dsrc, j0 & 31);
-                            const float d1 = __shfl_sync(0xffffffffu, dsrc, (j0 + 1) & 31);
-                            const float m0 = ex2_approx(fminf(cs_i - rc.cs[hh][j0], 0.f)) * d0;
-                            const float m1 = ex2_approx(fminf(cs_i - rc.cs[hh][j0 + 1], 0.f)) * d1;
-                            wv[e] = pack_bf16x2(bf16_lo(wv[e]) * m0, bf16_hi(wv[e]) * m1);
-                        }
-                        tmem_st32(s_col + 64 + half * 32, wv);
-                    }
-                    tmem_wait_st();
-                    tc_fence_before_sync();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bars + kSlotFull);
-                }
+                state_exact_stilde<KH>(p, bars, abort_flag, rc, w.s.b, w.s.tile, w.s.hs0, s_col, nh, r, lane);
                 ++nh;
             }
             __syncwarp();
@@ -1062,23 +1158,9 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bars + kRecEmpty + st);
-            if (hard) {
-                wait_bar(bars + kM3Done, nh & 1, abort_flag, p.status);
-                tc_fence_after_sync();
-#pragma unroll 1
-                for (int hh = 0; hh < KH; ++hh) {
-                    uint32_t v[64];
-                    const uint32_t a = tmem + lane_off + kColZ + (k & 1) * 128 + hh * 64;
-                    tmem_ld64_sync(a, v);
-                    const float zsh = (KH == 2 && hh) ? zs[KH - 1] : zs[0];
-#pragma unroll
-                    for (int q = 0; q < 64; ++q) v[q] = __float_as_uint(__uint_as_float(v[q]) * zsh);
-                    tmem_st64(a, v);
-                }
-                tmem_wait_st();
-                tc_fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bars + kZScaled);
+            if (__builtin_expect(hard, 0)) {
+                out_exact_scale<KH>(bars, abort_flag, p.status, tmem + lane_off + kColZ + (k & 1) * 128, zs[0],
+                                    zs[KH - 1], nh, lane);
                 ++nh;
             }
             wait_bar(bars + kZFull + (k & 1), (k >> 1) & 1, abort_flag, p.status);
@@ -1088,7 +1170,7 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             // once the last columns are in registers
             uint8_t* ys = sm + Smem::kC + st * 2 * kHalf + r * 128;
             const bool add_dx = hard && p.D;
-            if (!add_dx) {
+            if (__builtin_expect(!add_dx, 1)) {
 #pragma unroll 1
                 for (int j = 0; j < 2 * KH; ++j) {
                     const int hh = j >> 1, half = j & 1;
@@ -1116,47 +1198,8 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
                     }
                 }
             } else {
-#pragma unroll 1
-                for (int j = 0; j < 2 * KH; ++j) {
-                    const int hh = j >> 1, half = j & 1;
-                    uint32_t zv[32];
-                    tmem_ld32_sync(tmem + lane_off + kColZ + (k & 1) * 128 + hh * 64 + half * 32, zv);
-                    if (j == 2 * KH - 1) {
-                        tc_fence_before_sync();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(bars + kZEmpty + (k & 1));
-                    }
-                    const float eh = (KH == 2 && hh) ? e[KH - 1] : e[0];
-                    float dh = 0.f;
-                    if (add_dx) dh = __ldg(p.D + (cur.hs0 + hh) / p.sub);
-                    const uint4* xg = reinterpret_cast<const uint4*>(p.x + (row0 + hh) * kP + half * 32);
-#pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {
-                        float xv[8];
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) xv[u] = 0.f;
-                        if (add_dx && live) {
-                            // exact form: y = Z + D x, x from global memory
-                            const uint4 xq = __ldg(xg + c4);
-                            const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                xv[2 * u] = dh * bf16_lo(xw[u]);
-                                xv[2 * u + 1] = dh * bf16_hi(xw[u]);
-                            }
-                        }
-                        uint32_t o[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int i = 8 * c4 + 2 * u;
-                            o[u] = pack_bf16x2(fmaf(eh, __uint_as_float(zv[i]), xv[2 * u]),
-                                               fmaf(eh, __uint_as_float(zv[i + 1]), xv[2 * u + 1]));
-                        }
-                        const int c = 4 * half + c4;
-                        *reinterpret_cast<uint4*>(ys + hh * kHalf + (((c ^ r) & 7) << 4)) =
-                            make_uint4(o[0], o[1], o[2], o[3]);
-                    }
-                }
+                out_exact_epilogue<KH>(bars, tmem + lane_off + kColZ + (k & 1) * 128, ys, p.x, row0, p.D, cur.hs0,
+                                       p.sub, live, r, lane, k & 1);
             }
             fence_async_shared();
             __syncwarp();
