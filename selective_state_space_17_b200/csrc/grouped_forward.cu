@@ -406,6 +406,39 @@ struct Walker {
 // Exact-form tiles are rare; their parts of the role loops live out of line so
 // that the hot loops stay compact in the instruction cache.
 
+// MMA warp, exact form: once the raw X is in the H' buffer and the output
+// warps have scaled Z, one masked product per head (Z_h += S~_h X_h, S~_h from
+// TMEM as the state warps hand it over), then the tile's Z, S and H' buffers
+// are released.
+template <int KH>
+__device__ __noinline__ void mma_exact_products(uint64_t* bars, volatile int* abort_flag, unsigned int* status,
+                                                uint32_t zcol, uint32_t tmem, uint64_t dhp, uint32_t nh, int zb)
+{
+    constexpr uint32_t id_y1 = idesc_bf16(128, 64, false, true);
+    wait_bar(bars + kRawX, nh & 1, abort_flag, status);
+    wait_bar(bars + kZScaled, nh & 1, abort_flag, status);
+#pragma unroll 1
+    for (int hh = 0; hh < KH; ++hh) {
+        const uint32_t u = nh * KH + hh;
+        wait_bar(bars + kSlotFull, u & 1, abort_flag, status);
+        tc_fence_after_sync();
+        if (elect_one_sync()) {
+#pragma unroll 1
+            for (int q = 0; q < kT / 16; ++q)
+                mma_bf16_tmem_a(zcol + hh * 64, tmem + kColS + 64 + q * 8, dhp + ((hh * kHalf) >> 4) + q * (2048 >> 4),
+                                id_y1, true);
+            mma_commit(bars + kSlotFree);
+        }
+        __syncwarp();
+    }
+    if (elect_one_sync()) {
+        mma_commit(bars + kZFull + zb);
+        mma_commit(bars + kSFree);
+        mma_commit(bars + kHpEmpty);
+    }
+    __syncwarp();
+}
+
 // State warps: S~_h,ij = tril(S)_ij 2^(cs_i - cs_j) dt_j of each head into
 // columns 64-127 of the S buffer, handed to the MMA warp one head at a time.
 template <int KH>
@@ -670,7 +703,6 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
         // the recurrence from tile to tile, have their own issuing warp.)
         constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
         constexpr uint32_t id_y = idesc_bf16(128, 64 * KH, false, true);
-        constexpr uint32_t id_y1 = idesc_bf16(128, 64, false, true);
         const uint64_t dc0 = sdesc_sw128(smem_addr(sm + Smem::kC), 16, 1024);
         const uint64_t db0 = sdesc_sw128(smem_addr(sm + Smem::kB), 16, 1024);
         const uint64_t dx0 = sdesc_sw128(smem_addr(sm + Smem::kX), kHalf, 1024);   // X', MN-major
@@ -752,28 +784,7 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
                                     bars + kRawX);
                 }
                 __syncwarp();
-                wait_bar(bars + kRawX, nh & 1, abort_flag, p.status);
-                wait_bar(bars + kZScaled, nh & 1, abort_flag, p.status);
-#pragma unroll
-                for (int hh = 0; hh < KH; ++hh) {
-                    const uint32_t u = nh * KH + hh;
-                    wait_bar(bars + kSlotFull, u & 1, abort_flag, p.status);
-                    tc_fence_after_sync();
-                    if (elect_one_sync()) {
-#pragma unroll
-                        for (int q = 0; q < kT / 16; ++q)
-                            mma_bf16_tmem_a(zcol + hh * 64, tmem + kColS + 64 + q * 8,
-                                            dhp + ((hh * kHalf) >> 4) + q * (2048 >> 4), id_y1, true);
-                        mma_commit(bars + kSlotFree);
-                    }
-                    __syncwarp();
-                }
-                if (elect_one_sync()) {
-                    mma_commit(bars + kZFull + zb);
-                    mma_commit(bars + kSFree);
-                    mma_commit(bars + kHpEmpty);
-                }
-                __syncwarp();
+                mma_exact_products<KH>(bars, abort_flag, p.status, zcol, tmem, dhp, nh, zb);
                 ++nh;
             }
             if (elect_one_sync()) {
