@@ -7,11 +7,12 @@
 // "Mamba paper review" (youngju.dev), section 3.3.
 //
 // The step is bound by HBM: the fp32 state is read and written once (P*N*8
-// bytes per head) and everything else is small. One CTA of 8 warps per (b, h);
-// a warp owns whole state rows p and moves them with 128-bit accesses (lane l
-// holds n = 4l .. 4l+3 of each 128-column stripe), eight rows in flight per
-// warp (a whole 64 x 128 head's state per CTA, so that enough bytes are in
-// flight to cover the HBM latency), and reduces y_p with shuffles.
+// bytes per head) and everything else is small. A warp owns whole state rows p
+// and moves them with 128-bit accesses (lane l holds n = 4l .. 4l+3 of each
+// 128-column stripe), eight rows at a time, and reduces y_p with shuffles.
+// For N <= 128 persistent warps stream items of eight rows, each warp loading
+// the next item (state rows and every small operand) before it updates and
+// stores the current one; otherwise one CTA of 8 warps per (b, h).
 #include "common.cuh"
 
 namespace ssd {
@@ -100,6 +101,78 @@ step_vec(StepArgs a)
     }
 }
 
+// Streaming path: N <= 128, N % 4 == 0 (one 128-bit access per lane and state
+// row). Persistent warps walk items of eight rows of one head's state (a warp
+// owns whole rows, so y_p is a warp reduction); each warp loads the next
+// item's rows before it updates and stores the current ones, so that the
+// state stream has no gaps between items and no tail of partly filled waves.
+constexpr int kStreamCtasPerSm = 2;
+
+// One item's operands, loaded a whole item ahead of their use.
+struct StreamItem {
+    float4 h[kRowsInFlight];  // state rows p0 .. p0 + 7, columns 4 lane .. 4 lane + 3
+    float4 bq, cq;            // B and C at those columns
+    float xr[kRowsInFlight];  // x of the rows
+    float dt, A, D;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kWarps * 32, kStreamCtasPerSm)
+step_stream(StepArgs a, int items)
+{
+    const int lane = threadIdx.x & 31;
+    const int nwarps = gridDim.x * kWarps;
+    const int rb = (a.P + kRowsInFlight - 1) / kRowsInFlight;  // items per head
+    const bool lane_live = lane * 4 < a.N;
+    auto fetch = [&](int item, StreamItem& it) {
+        const int bh = item / rb, p0 = (item - bh * rb) * kRowsInFlight;
+        const int b = bh / a.H, h = bh % a.H, g = h / (a.H / a.G);
+        const float* st = a.state + ((size_t)bh * a.P + p0) * a.N + lane * 4;
+#pragma unroll
+        for (int r = 0; r < kRowsInFlight; ++r)
+            it.h[r] = (lane_live && p0 + r < a.P) ? __ldcs(reinterpret_cast<const float4*>(st + (size_t)r * a.N))
+                                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+        it.bq = it.cq = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (lane_live) {
+            it.bq = load4<T>(static_cast<const T*>(a.Bm) + ((size_t)b * a.G + g) * a.N + lane * 4);
+            it.cq = load4<T>(static_cast<const T*>(a.Cm) + ((size_t)b * a.G + g) * a.N + lane * 4);
+        }
+        const T* x = static_cast<const T*>(a.x) + (size_t)bh * a.P + p0;
+#pragma unroll
+        for (int r = 0; r < kRowsInFlight; ++r) it.xr[r] = p0 + r < a.P ? io<T>::load(x + r) : 0.f;
+        it.dt = a.dt[bh];
+        it.A = a.A[h];
+        it.D = a.D ? a.D[h] : 0.f;
+    };
+    int item = blockIdx.x * kWarps + (threadIdx.x >> 5);
+    StreamItem cur;
+    if (item < items) fetch(item, cur);
+    while (item < items) {
+        const int next = item + nwarps;
+        StreamItem nxt;
+        if (next < items) fetch(next, nxt);
+        const int bh = item / rb, p0 = (item - bh * rb) * kRowsInFlight;
+        const float decay = expf(cur.dt * cur.A);
+        T* y = static_cast<T*>(a.y) + (size_t)bh * a.P + p0;
+        float* st = a.state + ((size_t)bh * a.P + p0) * a.N + lane * 4;
+#pragma unroll
+        for (int r = 0; r < kRowsInFlight; ++r) {
+            if (p0 + r >= a.P) break;
+            const float u = cur.dt * cur.xr[r];
+            float4 v = cur.h[r];
+            v.x = decay * v.x + u * cur.bq.x;
+            v.y = decay * v.y + u * cur.bq.y;
+            v.z = decay * v.z + u * cur.bq.z;
+            v.w = decay * v.w + u * cur.bq.w;
+            const float s = warp_sum(v.x * cur.cq.x + v.y * cur.cq.y + v.z * cur.cq.z + v.w * cur.cq.w);
+            if (lane_live) __stcs(reinterpret_cast<float4*>(st + (size_t)r * a.N), v);
+            if (lane == 0) io<T>::store(y + r, s + cur.D * cur.xr[r]);
+        }
+        cur = nxt;
+        item = next;
+    }
+}
+
 // Scalar path: any N.
 template <typename T>
 __global__ void __launch_bounds__(kWarps * 32)
@@ -134,7 +207,12 @@ template <typename T>
 cudaError_t run(const StepArgs& a, const LaunchCtx& ctx)
 {
     const int grid = a.B * a.H;
-    if (a.N % 4 == 0)
+    if (a.N % 4 == 0 && a.N <= 128) {
+        const int items = a.B * a.H * ((a.P + kRowsInFlight - 1) / kRowsInFlight);
+        const int sms = ctx.num_sms > 0 ? ctx.num_sms : 1;
+        const int ctas = min((items + kWarps - 1) / kWarps, sms * kStreamCtasPerSm);
+        step_stream<T><<<ctas, kWarps * 32, 0, ctx.stream>>>(a, items);
+    } else if (a.N % 4 == 0)
         step_vec<T><<<grid, kWarps * 32, 0, ctx.stream>>>(a);
     else
         step_scalar<T><<<grid, kWarps * 32, 0, ctx.stream>>>(a);
