@@ -155,18 +155,49 @@ step_stream(StepArgs a, int items)
         const float decay = expf(cur.dt * cur.A);
         T* y = static_cast<T*>(a.y) + (size_t)bh * a.P + p0;
         float* st = a.state + ((size_t)bh * a.P + p0) * a.N + lane * 4;
+        float dot[kRowsInFlight];  // this lane's part of y_p for each row
 #pragma unroll
         for (int r = 0; r < kRowsInFlight; ++r) {
-            if (p0 + r >= a.P) break;
-            const float u = cur.dt * cur.xr[r];
+            const float u = cur.dt * cur.xr[r];  // 0 for rows past P
             float4 v = cur.h[r];
             v.x = decay * v.x + u * cur.bq.x;
             v.y = decay * v.y + u * cur.bq.y;
             v.z = decay * v.z + u * cur.bq.z;
             v.w = decay * v.w + u * cur.bq.w;
-            const float s = warp_sum(v.x * cur.cq.x + v.y * cur.cq.y + v.z * cur.cq.z + v.w * cur.cq.w);
-            if (lane_live) __stcs(reinterpret_cast<float4*>(st + (size_t)r * a.N), v);
-            if (lane == 0) io<T>::store(y + r, s + cur.D * cur.xr[r]);
+            dot[r] = v.x * cur.cq.x + v.y * cur.cq.y + v.z * cur.cq.z + v.w * cur.cq.w;
+            if (lane_live && p0 + r < a.P) __stcs(reinterpret_cast<float4*>(st + (size_t)r * a.N), v);
+        }
+        // the eight row sums in 9 shuffles instead of 40: at each step a lane
+        // keeps half of its rows and adds the partner's part of them, so after
+        // the 16-, 8- and 4-lane exchanges lane l holds row (l >> 2) & 7 (over
+        // its quad), and the 2- and 1-lane exchanges finish the sum
+        {
+            const bool hi16 = lane & 16, hi8 = lane & 8, hi4 = lane & 4;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float give = hi16 ? dot[i] : dot[i + 4];
+                const float keep = hi16 ? dot[i + 4] : dot[i];
+                dot[i] = keep + __shfl_xor_sync(0xffffffffu, give, 16);
+            }
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const float give = hi8 ? dot[i] : dot[i + 2];
+                const float keep = hi8 ? dot[i + 2] : dot[i];
+                dot[i] = keep + __shfl_xor_sync(0xffffffffu, give, 8);
+            }
+            {
+                const float give = hi4 ? dot[0] : dot[1];
+                const float keep = hi4 ? dot[1] : dot[0];
+                dot[0] = keep + __shfl_xor_sync(0xffffffffu, give, 4);
+            }
+            dot[0] += __shfl_xor_sync(0xffffffffu, dot[0], 2);
+            dot[0] += __shfl_xor_sync(0xffffffffu, dot[0], 1);
+            const int r = (hi16 ? 4 : 0) + (hi8 ? 2 : 0) + (hi4 ? 1 : 0);
+            float xr = cur.xr[0];
+#pragma unroll
+            for (int q = 1; q < kRowsInFlight; ++q)
+                if (r == q) xr = cur.xr[q];
+            if ((lane & 3) == 0 && p0 + r < a.P) io<T>::store(y + r, dot[0] + cur.D * xr);
         }
         cur = nxt;
         item = next;
