@@ -108,6 +108,20 @@ step_vec(StepArgs a)
 // state stream has no gaps between items and no tail of partly filled waves.
 constexpr int kStreamCtasPerSm = 2;
 
+// Division by a divisor fixed for the launch: with s = ceil(log2 d) and
+// m = ceil(2^(32 + s) / d) - 2^32, q = (hi32(n * m) + n) >> s, exact for
+// 0 <= n < 2^31 (the round-up method of Granlund and Montgomery, "Division by
+// invariant integers using multiplication", 1994).
+struct FastDiv {
+    uint32_t m, s;
+    __host__ explicit FastDiv(uint32_t d) : m(0), s(0)
+    {
+        while ((1ull << s) < d) ++s;
+        m = static_cast<uint32_t>(((1ull << (32 + s)) + d - 1) / d - (1ull << 32));
+    }
+    __device__ __forceinline__ uint32_t div(uint32_t n) const { return (__umulhi(n, m) + n) >> s; }
+};
+
 // One item's operands, loaded a whole item ahead of their use.
 struct StreamItem {
     float4 h[kRowsInFlight];  // state rows p0 .. p0 + 7, columns 4 lane .. 4 lane + 3
@@ -118,15 +132,15 @@ struct StreamItem {
 
 template <typename T>
 __global__ void __launch_bounds__(kWarps * 32, kStreamCtasPerSm)
-step_stream(StepArgs a, int items)
+step_stream(StepArgs a, int items, FastDiv by_rb, FastDiv by_h, FastDiv by_hpg)
 {
     const int lane = threadIdx.x & 31;
     const int nwarps = gridDim.x * kWarps;
     const int rb = (a.P + kRowsInFlight - 1) / kRowsInFlight;  // items per head
     const bool lane_live = lane * 4 < a.N;
     auto fetch = [&](int item, StreamItem& it) {
-        const int bh = item / rb, p0 = (item - bh * rb) * kRowsInFlight;
-        const int b = bh / a.H, h = bh % a.H, g = h / (a.H / a.G);
+        const int bh = by_rb.div(item), p0 = (item - bh * rb) * kRowsInFlight;
+        const int b = by_h.div(bh), h = bh - b * a.H, g = by_hpg.div(h);
         const float* st = a.state + ((size_t)bh * a.P + p0) * a.N + lane * 4;
 #pragma unroll
         for (int r = 0; r < kRowsInFlight; ++r)
@@ -151,7 +165,7 @@ step_stream(StepArgs a, int items)
         const int next = item + nwarps;
         StreamItem nxt;
         if (next < items) fetch(next, nxt);
-        const int bh = item / rb, p0 = (item - bh * rb) * kRowsInFlight;
+        const int bh = by_rb.div(item), p0 = (item - bh * rb) * kRowsInFlight;
         const float decay = expf(cur.dt * cur.A);
         T* y = static_cast<T*>(a.y) + (size_t)bh * a.P + p0;
         float* st = a.state + ((size_t)bh * a.P + p0) * a.N + lane * 4;
@@ -238,11 +252,13 @@ template <typename T>
 cudaError_t run(const StepArgs& a, const LaunchCtx& ctx)
 {
     const int grid = a.B * a.H;
-    if (a.N % 4 == 0 && a.N <= 128) {
-        const int items = a.B * a.H * ((a.P + kRowsInFlight - 1) / kRowsInFlight);
+    const long long stream_items = static_cast<long long>(a.B) * a.H * ((a.P + kRowsInFlight - 1) / kRowsInFlight);
+    if (a.N % 4 == 0 && a.N <= 128 && stream_items < (1ll << 30)) {  // item indices stay below 2^31
+        const int items = static_cast<int>(stream_items);
         const int sms = ctx.num_sms > 0 ? ctx.num_sms : 1;
         const int ctas = min((items + kWarps - 1) / kWarps, sms * kStreamCtasPerSm);
-        step_stream<T><<<ctas, kWarps * 32, 0, ctx.stream>>>(a, items);
+        step_stream<T><<<ctas, kWarps * 32, 0, ctx.stream>>>(
+            a, items, FastDiv((a.P + kRowsInFlight - 1) / kRowsInFlight), FastDiv(a.H), FastDiv(a.H / a.G));
     } else if (a.N % 4 == 0)
         step_vec<T><<<grid, kWarps * 32, 0, ctx.stream>>>(a);
     else
