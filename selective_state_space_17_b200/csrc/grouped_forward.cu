@@ -61,8 +61,11 @@
 //   warps 4-7     state and mask: h_prev -> H' and the scaled h, piece
 //                 hand-off and final state; then S -> tril(S) (exact form:
 //                 S~_h per head)
-//   warps 8-11    output: y = e Z stored from registers (exact form: the row
-//                 scaling of Z first, and y = Z + D x)
+//   warps 8-11    output: y = e Z staged in the tile's C buffer and stored by
+//                 TMA (exact form: the row scaling of Z first, and y = Z + D x)
+// The exact-form parts of warps 1, 4-7 and 8-11 are out-of-line functions: it
+// is rare, and the hot loops of all roles together already miss in the SM's
+// instruction cache, so code in them that never runs still costs time.
 //   warps 12-15   scale: X' in place and Z's initial value
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -1143,8 +1146,9 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
         // Thread r owns token row r of the tile. Scaled form: Z started from
         // D x / e, so y = e Z. Exact form: Z_r *= 2^(cs_r) first, which the
         // per-head masked products then add to, and y = Z + D x with x read
-        // from global memory. Each row of y (128 bytes per head) is stored
-        // from registers; rows past L are not written.
+        // from global memory. Row r of y (128 bytes per head) goes into the
+        // tile's C buffer in the 128-byte swizzle, and one TMA store per head
+        // writes the tile (rows past L are clipped).
         const int wq = warp - kWgOut;
         const int r = wq * 32 + lane;  // token row i = TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
