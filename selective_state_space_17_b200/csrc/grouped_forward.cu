@@ -665,6 +665,17 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             const int st = k & 1;
             const uint32_t par = ((k >> 1) & 1) ^ 1;
             const int t0 = s.tile * kT;
+            // X first: its stage frees when MMA2 and the states product have
+            // read it, the C/B stage only once y, staged in C, is stored
+            wait_bar(bars + kEmptyX + st, par, abort_flag, p.status);
+            if (elect_one_sync()) {
+                mbar_arrive_expect_tx(bars + kFullX + st, KH * kHalf);
+#pragma unroll
+                for (int hh = 0; hh < KH; ++hh)
+                    tma_load_4d(sm + Smem::kX + st * 2 * kHalf + hh * kHalf, &tmX, 0, s.hs0 + hh, t0, s.b,
+                                bars + kFullX + st);
+            }
+            __syncwarp();
             wait_bar(bars + kEmptyCB + st, par, abort_flag, p.status);
             if (elect_one_sync()) {
                 mbar_arrive_expect_tx(bars + kFullCB + st, p.nkh * 2 * kHalf);
@@ -674,15 +685,6 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
                     tma_load_4d(sm + Smem::kB + st * 2 * kHalf + q * kHalf, &tmB, q * 64, s.g, t0, s.b,
                                 bars + kFullCB + st);
                 }
-            }
-            __syncwarp();
-            wait_bar(bars + kEmptyX + st, par, abort_flag, p.status);
-            if (elect_one_sync()) {
-                mbar_arrive_expect_tx(bars + kFullX + st, KH * kHalf);
-#pragma unroll
-                for (int hh = 0; hh < KH; ++hh)
-                    tma_load_4d(sm + Smem::kX + st * 2 * kHalf + hh * kHalf, &tmX, 0, s.hs0 + hh, t0, s.b,
-                                bars + kFullX + st);
             }
             __syncwarp();
             ++k;
