@@ -819,6 +819,9 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             const int st = k & 1;
             const uint32_t par = (k >> 1) & 1;
             const uint64_t stage = static_cast<uint64_t>(st * 2 * kHalf) >> 4;
+            // B of this tile has landed (the states product reads it; nothing
+            // else that this warp waits for implies it: X' only needs X)
+            wait_bar(bars + kFullCB + st, par, abort_flag, p.status);
             wait_bar(bars + kXpFull + st, par, abort_flag, p.status);
             wait_bar(bars + kHReady, k & 1, abort_flag, p.status);
             tc_fence_after_sync();
