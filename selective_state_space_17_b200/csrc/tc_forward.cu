@@ -190,7 +190,7 @@ enum Bar : int {
     kFullCB = 0,      // 2
     kEmptyCB = 2,     // 2 (two arrivals: after states, after MMA3)
     kFullX = 4,       // 3
-    kEmptyX = 7,      // 3
+    kEmptyX = 7,      // 3 (two arrivals: stream B's products and the w o X pass; one in mode 1)
     kFullXt = 10,
     kEmptyXt = 11,
     kFullRec = 12,    // 4
@@ -295,6 +295,7 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             mbar_init(bars + i, (i >= kEmptyRec && i < kEmptyRec + kCsStages) ? (states_only ? 1u : 5u)
                                 : (i >= kFullSt && i < kFullSt + 2)          ? 4u
                                 : (i >= kEmptyCB && i < kEmptyCB + 2)        ? (states_only ? 1u : 2u)
+                                : (i >= kEmptyX && i < kEmptyX + kXStages)   ? (states_only ? 1u : 2u)
                                                                              : 1u);
         mbar_fence_init();
         *abort_flag = 0;
@@ -574,7 +575,9 @@ tc_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             named_bar_sync(kBarPrep, 64);
             if (t == 0) {
                 mbar_arrive(bars + kFullXt);
-                if (states_only) mbar_arrive(bars + kEmptyX + xs);
+                // the X stage is free once w o X has read it as well: stream B's
+                // products finishing first does not mean this read is done
+                mbar_arrive(bars + kEmptyX + xs);
             }
         }
     } else if (warp >= kWgMask0 && warp < kWgMask0 + 4 && !states_only) {
