@@ -1101,8 +1101,7 @@ grouped_forward_kernel(const __grid_constant__ CUtensorMap tmX,
             }
 
             // ---- mask of tile k: S -> tril(S), as bf16 pairs over the first 64
-            // columns of the S buffer (block jb of 32 fp32 columns lands on
-            // columns 16 jb .. 16 jb + 15, which are already read)
+            // columns of the S buffer
             wait_bar(bars + kSFull, k & 1, abort_flag, p.status);
             tc_fence_after_sync();
             const uint32_t s_col = tmem + lane_off + kColS;
